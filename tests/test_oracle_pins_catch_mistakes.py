@@ -1,0 +1,143 @@
+"""The pins are sharp: plausible mistakes planted in the oracle (on the CPU,
+never in the CUDA path) make at least one pin fail.
+
+Each case swaps one oracle function for a mutated copy and checks that the
+corresponding pin would reject it.
+"""
+import itertools
+import json
+import os
+
+import ml_dtypes
+import numpy as np
+
+import oracle
+from oracle import E4M3
+from oracle import fp8 as fp8_mod
+from oracle import prune as prune_mod
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                     "hand_worked_examples.json")))
+
+
+def _midpoint_pin(encode):
+    return all(encode(np.array([v], np.float32), E4M3)[0] == int(c, 16)
+               for v, c in GOLDEN["rne_midpoints"][E4M3])
+
+
+def test_ties_away_from_zero_is_caught():
+    def encode_ties_away(t, fmt):
+        table = oracle.decode_table(fmt)
+        top = oracle.max_code(fmt)
+        pos = table[: top + 1]
+        a = np.abs(t.astype(np.float64))
+        hi = np.minimum(np.searchsorted(pos, a), top)
+        lo = np.maximum(hi - 1, 0)
+        mag = np.where(pos[hi] - a <= a - pos[lo], hi, lo)   # ties go up
+        mag = np.where(a >= pos[top], top, mag)
+        return (mag | (np.signbit(t).astype(np.int64) << 7)).astype(np.uint8)
+    assert _midpoint_pin(oracle.encode_rne_sat)
+    assert not _midpoint_pin(encode_ties_away)
+
+
+def test_nonsaturating_cast_is_caught():
+    def encode_lib(t, fmt):
+        return np.asarray(t, np.float32).astype(ml_dtypes.float8_e4m3fn).view(np.uint8)
+    assert not _midpoint_pin(encode_lib)      # 1000 -> NaN instead of 448
+
+
+def _brute_force_compress_pin(compress):
+    codes = [0x00, 0x80, 0x01, 0x81, 0x38, 0xB8, 0x40, 0xC0]
+    groups = np.array(list(itertools.product(codes, repeat=4)), dtype=np.uint8)
+    vals, nib = compress(groups, E4M3)
+    mags = np.abs(groups.view(ml_dtypes.float8_e4m3fn).astype(np.float64))
+    for r in range(groups.shape[0]):
+        order = sorted(range(4), key=lambda j: (-mags[r, j], j))
+        i0, i1 = sorted(order[:2])
+        if nib[r, 0] != (i0 | (i1 << 2)):
+            return False
+    return True
+
+
+def test_tie_to_higher_index_is_caught(monkeypatch):
+    assert _brute_force_compress_pin(oracle.compress_24)
+
+    def ranks_high(mag):
+        r = np.zeros(mag.shape, dtype=np.int64)
+        for j in range(4):
+            for i in range(4):
+                if i != j:
+                    r[..., j] += (mag[..., i] > mag[..., j])
+                    if i > j:
+                        r[..., j] += (mag[..., i] == mag[..., j])
+        return r
+    import oracle.compress as comp
+    monkeypatch.setattr(comp, "group_ranks", ranks_high)
+    assert not _brute_force_compress_pin(comp.compress_24)
+
+
+def test_negative_zero_ranked_by_code_is_caught(monkeypatch):
+    import oracle.compress as comp
+    real_decode = comp.decode
+    # a mistake: rank by the raw byte, so 0x80 (-0.0) looks large
+    monkeypatch.setattr(comp, "decode", lambda codes, fmt: np.asarray(codes, np.float64))
+    assert not _brute_force_compress_pin(comp.compress_24)
+    monkeypatch.setattr(comp, "decode", real_decode)
+
+
+def test_swapped_nibble_fields_are_caught():
+    g = GOLDEN["compress_groups_e4m3"][1]
+    q = np.array([[int(c, 16) for c in g["codes"]]], dtype=np.uint8)
+    vals, nib = oracle.compress_24(q, E4M3)
+    swapped = ((nib & 3) << 2) | (nib >> 2)
+    assert nib[0, 0] == int(g["nibble"], 16)
+    assert swapped[0, 0] != int(g["nibble"], 16)
+
+
+def test_dropped_term_in_linear_is_caught():
+    g = GOLDEN["dot_product_e4m3"]
+    a = np.array([[int(c, 16) for c in g["a_codes"]]], dtype=np.uint8)
+    wq = oracle.encode_rne_sat(np.array(g["w_dense_values"], np.float32)[None, :], E4M3)
+    vals, nib = oracle.compress_24(wq, E4M3)
+    s = np.array([g["s_a"]], np.float32)
+    y, _, _ = oracle.sparse_linear_ref(a, E4M3, s, vals, nib, E4M3, s)
+    assert y[0, 0] == g["y_exact"]
+    # drop the second kept slot of every group
+    vals_half = vals.copy()
+    vals_half[:, 1::2] = 0
+    y2, _, _ = oracle.sparse_linear_ref(a, E4M3, s, vals_half, nib, E4M3, s)
+    assert y2[0, 0] != g["y_exact"]
+    # transposed scales (s_w applied per row m) on a 2x2 case change the result
+    a2 = np.vstack([a, a])
+    vals2, nib2 = np.vstack([vals, vals]), np.vstack([nib, nib])
+    sa2 = np.array([1.0, 2.0], np.float32)
+    sw2 = np.array([1.0, 4.0], np.float32)
+    y_ok, _, _ = oracle.sparse_linear_ref(a2, E4M3, sa2, vals2, nib2, E4M3, sw2)
+    y_tr, _, _ = oracle.sparse_linear_ref(a2, E4M3, sw2, vals2, nib2, E4M3, sa2)
+    assert not np.array_equal(y_ok, y_tr.T) or not np.array_equal(y_ok, y_tr)
+
+
+def _prune_pin(prune):
+    vals = [0.0, -0.0, 1.0, -1.0, 2.0, 0.5]
+    groups = np.array(list(itertools.product(vals, repeat=4)), dtype=np.float32)
+    out = prune(groups)
+    for r in range(groups.shape[0]):
+        order = sorted(range(4), key=lambda j: (-abs(float(groups[r, j])), j))
+        keep = set(order[:2])
+        for j in range(4):
+            want = groups[r, j] if j in keep else np.float32(0.0)
+            if out[r, j].view(np.uint32) != np.float32(want).view(np.uint32):
+                return False
+    return True
+
+
+def test_prune_mistakes_are_caught(monkeypatch):
+    assert _prune_pin(oracle.prune_24)
+    real = prune_mod.group_ranks
+    monkeypatch.setattr(prune_mod, "group_ranks", lambda m: 3 - real(m))   # keeps the smallest
+    assert not _prune_pin(prune_mod.prune_24)
+    monkeypatch.setattr(prune_mod, "group_ranks", real)
+    # dropped entries written as -0.0 instead of +0.0
+    monkeypatch.setattr(prune_mod, "prune_24", lambda w: np.where(
+        real(np.abs(w.reshape(-1, 1, 4)).astype(np.float64)).reshape(w.shape) < 2, w, np.float32(-0.0)))
+    assert not _prune_pin(prune_mod.prune_24)
