@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the row-wise scaled 2:4 sparse FP8 linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--m 16] [--impl ours|reference]
+
+Workload: the Llama-3.1-8B MLP gate/up projection at decode (K=4096,
+N=14336, M in {1, 4, 16}; the headline line uses M=16), synthetic seeded
+inputs (A ~ N(0,1) bf16, W ~ N(0, 0.02) bf16, magnitude-pruned 2:4, both
+quantised row-wise to e4m3, no bias).
+
+A step is one forward of the layer: dynamic row-wise FP8 quantisation of the
+activation followed by the sparse FP8 GEMM with its scale epilogue.  The
+weight is prepared once before timing (prune -> quantise -> compress), as the
+layer does at load time; those kernels are timed separately under "offline".
+The metric's unit for this memory-bound shape is GB/s of compressed weight
+bytes (kept values + metadata) per step.
+
+Timing: W eager warm-up steps, then exactly K steps captured in one CUDA
+graph and replayed once between CUDA events on the launching stream, with a
+barrier and a device synchronise on both sides; the max over ranks is
+reported.  The K steps rotate over 8 copies of the compressed weight
+(8 x 36.7 MB > the 126 MB L2), so no step finds its weight in L2.  Under
+torchrun every rank runs an independent replica (weak scaling, no data-path
+collective).
+
+`--impl reference` times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2:4 FP8 rowwise sparse linear TFLOP/s & GB/s, % roofline, M=1..8192"
+WORKLOAD = "decode_gate_up_8b"
+M_TO_SHAPE = {1: 0, 4: 1, 16: 2}
+K_DIM, N_DIM = 4096, 14336
+WEIGHT_COPIES = 8
+L2_NOTE = "rotating 8 copies of the compressed weight (8 x 36.7 MB > 126 MB L2)"
+
+# ncu DRAM traffic (read + write bytes) of one sparse-GEMM launch at M=16,
+# valid only for the kernel source it was measured on.
+NCU_TRAFFIC = {"sha1": None, "bytes_per_launch": None}
+
+
+def compressed_weight_bytes(n, k):
+    npad = ((n + 127) // 128) * 128
+    return npad * k // 2 + npad * k // 8
+
+
+def gemm_algorithmic_bytes(m, n, k):
+    """HBM bytes one GEMM launch must move: compressed weight + metadata,
+    weight scales, activation codes and scales, bf16 output."""
+    return compressed_weight_bytes(n, k) + 4 * n + m * k + 4 * m + 2 * m * n
+
+
+def kernel_source_sha1():
+    p = os.path.join(ROOT, "semi_structured_sparse_rowwise_b200", "csrc", "sparse_linear.cuh")
+    with open(p, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    def __init__(self, device_index, period_s=0.002):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+            return self
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
+        return self
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        names = {
+            0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown",
+            0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown",
+        }
+        for bit, name in names.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._thr.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(backend):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, local, world
+
+
+def dist_max(value, world, device=None):
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_step_rate(m, seconds=10.0, n_sample=512):
+    """Oracle throughput on a bounded sample of the decode step: quantise the
+    activation (all m rows) and compute n_sample output columns, repeated for
+    about `seconds`.  Returns (GB/s of compressed weight bytes, cores, note)."""
+    import numpy as np
+    import oracle
+    from semi_structured_sparse_rowwise_b200 import synthetic
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    key = (m, n_sample)
+    if key not in _ORACLE_INPUTS:
+        x_bits, w_bits, _, _ = synthetic.workload_inputs(WORKLOAD, M_TO_SHAPE[m])
+        cols = np.arange(n_sample)
+        w32 = oracle.bf16_bits_to_f32(w_bits[cols])
+        wq, sw = oracle.quantize_rowwise(oracle.prune_24(w32), "e4m3")
+        vals, nib = oracle.compress_24(wq, "e4m3")
+        _ORACLE_INPUTS[key] = (oracle.bf16_bits_to_f32(x_bits), vals, nib, sw)
+    x32, vals, nib, sw = _ORACLE_INPUTS[key]
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        aq, sa = oracle.quantize_rowwise(x32, "e4m3")
+        oracle.sparse_linear_ref(aq, "e4m3", sa, vals, nib, "e4m3", sw)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    # one sample covers n_sample of the N output columns: scale the work
+    frac = n_sample / N_DIM
+    step_time = dt / reps / frac
+    rate = compressed_weight_bytes(N_DIM, K_DIM) / step_time / 1e9
+    note = ("oracle (numpy fp64) quantise of the %dx%d activation + linear for %d of %d "
+            "output columns, %d repetitions in %.1f s, scaled to the full N"
+            % (m, K_DIM, n_sample, N_DIM, reps, dt))
+    return rate, cores, note, step_time
+
+
+def run_reference(args):
+    rank, local, world = dist_setup("gloo")
+    if rank != 0:
+        return 0
+    m = args.m
+    # each step: a bounded sample of the workload (the oracle is slow); the
+    # whole run stays around a minute whatever K and W are
+    per_step_s = min(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_step_rate(m, seconds=per_step_s)
+    rates, step_times = [], []
+    note = ""
+    cores = 1
+    for _ in range(args.steps):
+        r, cores, note, st = oracle_step_rate(m, seconds=per_step_s)
+        rates.append(r)
+        step_times.append(st)
+    value = statistics.mean(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(step_times) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "m": m, "k": K_DIM, "n": N_DIM, "a_dtype": "e4m3",
+                   "w_dtype": "e4m3", "bias": False},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": note},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU path
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    rank, local, world = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import semi_structured_sparse_rowwise_b200 as S
+    from semi_structured_sparse_rowwise_b200 import synthetic
+
+    S.load_library()
+    m = args.m
+    x_bits, w_bits, _, seeds = synthetic.workload_inputs(WORKLOAD, M_TO_SHAPE[m])
+    n, k = w_bits.shape
+    stream = torch.cuda.current_stream(dev)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    w_dev = bf16(w_bits)
+    x_dev = bf16(x_bits)
+
+    # ---- offline weight preparation (timed separately)
+    def prep():
+        wp = S.sfp8_prune_24(w_dev)
+        wq, sw = S.sfp8_quantize_rowwise(wp, "e4m3")
+        vals, meta = S.sfp8_compress_24(wq, "e4m3")
+        return wp, wq, sw, vals, meta
+
+    wp, wq, sw, vals, meta = prep()
+    torch.cuda.synchronize(dev)
+    off = {}
+    for name, fn in (("prune_24", lambda: S.sfp8_prune_24(w_dev, out=wp)),
+                     ("quantize_weight", lambda: S.sfp8_quantize_rowwise(wp, "e4m3", q=wq, scales=sw)),
+                     ("compress_24", lambda: S.sfp8_compress_24(wq, "e4m3", values=vals, meta=meta))):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        off[name] = e0.elapsed_time(e1) / reps
+    wbytes_bf16 = n * k * 2
+    off_gbs = {
+        "prune_24": {"ms": off["prune_24"], "GB/s": 2 * wbytes_bf16 / off["prune_24"] / 1e6},
+        "quantize_weight": {"ms": off["quantize_weight"],
+                            "GB/s": (wbytes_bf16 + n * k + 4 * n) / off["quantize_weight"] / 1e6},
+        "compress_24": {"ms": off["compress_24"],
+                        "GB/s": (n * k + compressed_weight_bytes(n, k)) / off["compress_24"] / 1e6},
+    }
+
+    # ---- the step's buffers
+    copies = [(vals.clone(), meta.clone(), sw.clone()) for _ in range(WEIGHT_COPIES)]
+    del vals, meta
+    aq = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    sa = torch.empty((m,), dtype=torch.float32, device=dev)
+    ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(WEIGHT_COPIES)]
+    ws = S.new_workspace(m, n, k, dev)
+
+    def quantize():
+        S.sfp8_quantize_rowwise(x_dev, "e4m3", q=aq, scales=sa)
+
+    def gemm(j):
+        v, mt, s = copies[j % WEIGHT_COPIES]
+        S.sfp8_sparse_linear(aq, "e4m3", sa, v, mt, "e4m3", s, n, k, out=ys[j % WEIGHT_COPIES],
+                             workspace=ws)
+
+    def step(j):
+        quantize()
+        gemm(j)
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize(dev)
+
+    def capture(fn, count):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for j in range(count):
+                    fn(j)
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        return g
+
+    def timed(g, sampler=None):
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        e1.synchronize()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        return e0.elapsed_time(e1)
+
+    steps = args.steps
+    g_step = capture(step, steps)
+    g_step.replay()                      # untimed: graph upload
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        ms = timed(g_step)
+    ms = dist_max(ms, world, dev)
+    clocks = clk.summary()
+    wbytes = compressed_weight_bytes(n, k)
+    value = world * wbytes * steps / (ms * 1e-3) / 1e9
+
+    # ---- the dominant kernel alone (sparse GEMM), same rotation
+    quantize()
+    g_gemm = capture(gemm, steps)
+    g_gemm.replay()
+    torch.cuda.synchronize(dev)
+    ms_gemm = dist_max(timed(g_gemm), world, dev)
+    gemm_us = ms_gemm * 1e3 / steps
+    g_q = capture(lambda j: quantize(), steps)
+    g_q.replay()
+    ms_q = dist_max(timed(g_q), world, dev)
+    peak, peak_kind = measured_peaks()
+    alg = gemm_algorithmic_bytes(m, n, k)
+    achieved = alg / (gemm_us * 1e-6) / 1e9
+    traffic = None
+    if NCU_TRAFFIC["sha1"] == kernel_source_sha1():
+        traffic = NCU_TRAFFIC["bytes_per_launch"]
+
+    # ---- end to end through the layer, host buffers, eager calls
+    layer = S.SparseFp8Linear.from_compressed(copies[0][0], copies[0][1], copies[0][2], n, k)
+    x_host = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(
+        torch.bfloat16).pin_memory()
+    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+    x_stage = torch.empty((m, k), dtype=torch.bfloat16, device=dev)
+    for _ in range(max(3, args.warmup)):
+        layer.forward_host(x_host, y_host, x_dev=x_stage, y_dev=ys[0])
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        layer.forward_host(x_host, y_host, x_dev=x_stage, y_dev=ys[0])
+    e1.record()
+    e1.synchronize()
+    ms_e2e = dist_max(e0.elapsed_time(e1), world, dev)
+    barrier(world)
+    e2e = {"value": world * wbytes * steps / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2,
+           "ms_per_step": ms_e2e / steps,
+           "path": "SparseFp8Linear.forward_host (eager calls, pinned host buffers)"}
+
+    # ---- the other decode batch sizes (context lines, same method)
+    per_m = {}
+    if args.all_m and world == 1:
+        for m2 in (1, 4, 16):
+            if m2 == m:
+                continue
+            x2 = bf16(synthetic.workload_inputs(WORKLOAD, M_TO_SHAPE[m2])[0])
+            aq2 = torch.empty((m2, k), dtype=torch.uint8, device=dev)
+            sa2 = torch.empty((m2,), dtype=torch.float32, device=dev)
+            y2 = torch.empty((m2, n), dtype=torch.bfloat16, device=dev)
+            ws2 = S.new_workspace(m2, n, k, dev)
+
+            def step2(j, x2=x2, aq2=aq2, sa2=sa2, y2=y2, ws2=ws2, m2=m2):
+                S.sfp8_quantize_rowwise(x2, "e4m3", q=aq2, scales=sa2)
+                v, mt, s = copies[j % WEIGHT_COPIES]
+                S.sfp8_sparse_linear(aq2, "e4m3", sa2, v, mt, "e4m3", s, n, k, out=y2,
+                                     workspace=ws2)
+            for j in range(args.warmup):
+                step2(j)
+            g2 = capture(step2, steps)
+            g2.replay()
+            ms2 = timed(g2)
+            per_m[str(m2)] = {"value": wbytes * steps / (ms2 * 1e-3) / 1e9, "unit": "GB/s",
+                              "ms_per_step": ms2 / steps}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "m": m, "k": k, "n": n, "a_dtype": "e4m3",
+                   "w_dtype": "e4m3", "bias": False, "l2": L2_NOTE,
+                   "step": "sfp8_quantize_rowwise + sfp8_sparse_linear",
+                   "weight_bytes_per_step": wbytes, "seeds": seeds,
+                   "parallelism": "replica" if world > 1 else "single"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "sparse_linear_kernel<16>" if m <= 16 else "sparse_linear_kernel",
+                     "algorithmic_bytes_per_launch": alg, "us_per_launch": gemm_us,
+                     "peak_source": peak_kind + " hbm_gbs (MEASURED_PEAKS.json)"},
+        "quantize_us_per_launch": ms_q * 1e3 / steps,
+        "e2e": e2e,
+        "gpu_launches": 2 * steps,
+        "clocks": clocks,
+        "offline": off_gbs,
+    }
+    if per_m:
+        line["per_m"] = per_m
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, note, _ = oracle_step_rate(m, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": note}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g_step, g_gemm, g_q
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--all-m", action="store_true", help="also time M=1 and M=4")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,203 @@
+/*
+ * sfp8 -- row-wise scaled 2:4 sparse FP8 linear layer for B200 (sm_100a).
+ *
+ * C ABI of libsfp8.so.  Plain pointers and sizes only; no C++ or framework
+ * types cross this boundary.  Every pointer argument named *device* must be
+ * device memory of the current CUDA device; the caller owns every buffer.
+ *
+ * The operation (page "Add CUTLASS-based row-wise scaled sparse FP8 kernel",
+ * pytorch/ao pull request 1671, items 1, 3 and 4):
+ *
+ *     y[m, n] = s_a[m] * s_w[n] * sum_k A_q[m, k] * W_q[n, k]  (+ bias[n])
+ *
+ * where A_q, s_a come from dynamic per-row FP8 quantisation of the
+ * activation, and W_q, s_w from the same quantisation of a 2:4-pruned weight
+ * that is then stored compressed (kept values + 2-bit index metadata).
+ *
+ * Conventions shared by all entry points:
+ *  - Asynchronous: work is enqueued on `stream` (a cudaStream_t; NULL means
+ *    the legacy default stream).  Nothing is synchronised.
+ *  - Validation errors are returned synchronously before anything is
+ *    launched: null pointers, unsupported shapes or dtypes, misalignment,
+ *    a too-small workspace, a device that is not sm_100.  A failed launch
+ *    returns SFP8_ERR_CUDA.  No exception crosses the ABI.
+ *  - Device-side failures (a pipeline wait that ran out its time limit) are
+ *    recorded in a per-device status word; read it with
+ *    sfp8_read_device_status() after synchronising.
+ *  - Reentrant: independent calls may run concurrently on different streams
+ *    as long as they do not share an output or a workspace.
+ *  - Deterministic: the same inputs give bit-identical outputs, run to run.
+ *  - Empty problems (rows, m or n equal to 0) return SFP8_OK and launch
+ *    nothing.
+ *  - Strides (ld) are in elements.  Row-major everywhere.
+ */
+#ifndef SFP8_H_
+#define SFP8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SFP8_OK = 0,
+  SFP8_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum  */
+  SFP8_ERR_UNSUPPORTED_SHAPE = 2,  /* e.g. k not a multiple of 128           */
+  SFP8_ERR_MISALIGNED = 3,         /* a base pointer or stride not aligned   */
+  SFP8_ERR_UNSUPPORTED_DTYPE = 4,  /* dtype not accepted by this entry point */
+  SFP8_ERR_ARCH = 5,               /* current device is not sm_100           */
+  SFP8_ERR_WORKSPACE = 6,          /* workspace missing or too small         */
+  SFP8_ERR_CUDA = 7,               /* a CUDA runtime/driver call failed      */
+  SFP8_ERR_TIMEOUT = 8,            /* a device-side wait hit its time limit  */
+  SFP8_ERR_DEVICE_CHECK = 9        /* a device-side consistency check failed */
+} sfp8_status;
+
+typedef enum {
+  SFP8_BF16 = 0,
+  SFP8_F16 = 1,
+  SFP8_F32 = 2,
+  SFP8_E4M3 = 3,  /* OCP e4m3 ("e4m3fn"): max 448, no infinities   */
+  SFP8_E5M2 = 4   /* OCP e5m2: max 57344                          */
+} sfp8_dtype;
+
+/* Bits of the device status word. */
+#define SFP8_DEVICE_TIMEOUT     0x1u  /* a bounded mbarrier wait gave up     */
+#define SFP8_DEVICE_CHECK_FAIL  0x2u  /* a device-side check failed          */
+
+/* Version of the compressed-weight layout written by sfp8_compress_24. */
+#define SFP8_LAYOUT_VERSION 1
+
+/*
+ * Dynamic row-wise FP8 quantisation (the activation path of item 4; also
+ * used once on the pruned weight).  For each row r of x:
+ *     amax     = max_c |x[r, c]|                     (fp32, exact)
+ *     s        = max(amax, 1e-12f) / FP8_MAX         (IEEE fp32 division)
+ *     q[r, c]  = RNE_satfinite_fp8(x[r, c] / s)      (IEEE fp32 division,
+ *                                                      then one rounding)
+ * FP8_MAX = 448 (E4M3) or 57344 (E5M2).  Overflow saturates; the sign of a
+ * value that rounds to zero is kept.  NaN/Inf inputs are outside the
+ * contract.
+ *
+ *  x       device, [rows, cols] of x_dtype (BF16, F16 or F32), row stride
+ *          ld_x >= cols elements; 16-byte aligned base, ld_x*size 16-byte
+ *          multiple.
+ *  q       device, [rows, cols] bytes (q_dtype E4M3 or E5M2), row stride
+ *          cols; 16-byte aligned.
+ *  scales  device, [rows] float32 (s above); 4-byte aligned.
+ *  cols % 16 == 0 (cols may be 0: scales are then the guard scale).
+ */
+sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype,
+                                  int64_t rows, int64_t cols, int64_t ld_x,
+                                  void* q, sfp8_dtype q_dtype, float* scales,
+                                  void* stream);
+
+/*
+ * 2:4 magnitude pruning along the row (the weight preparation that the
+ * page's "sparsify/quantize method" performs before quantisation): in every
+ * group of four consecutive elements keep the two of largest |w| (-0.0 is
+ * zero; ties to the lower index) and write +0.0 in the other two.  Kept
+ * elements are copied bit for bit.
+ *
+ *  w       device, [rows, cols] of dtype (BF16, F16 or F32), row stride ld;
+ *          16-byte aligned base, ld*size 16-byte multiple.
+ *  out     device, [rows, cols] of dtype, row stride cols, 16-byte aligned.
+ *          May not alias w unless ld == cols (then in-place is allowed).
+ *  cols % 16 == 0.
+ */
+sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows,
+                          int64_t cols, int64_t ld, void* out, void* stream);
+
+/*
+ * Compressed-weight sizes for an [n, k] FP8 weight (k % 128 == 0).
+ * Rows are padded to n_pad = ceil(n / 128) * 128.
+ *   values: n_pad * k / 2 bytes;  meta: n_pad * k / 8 bytes.
+ */
+int64_t sfp8_padded_rows(int64_t n);
+size_t sfp8_compressed_values_bytes(int64_t n, int64_t k);
+size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k);
+
+/*
+ * 2:4 compression of an FP8 weight (item 1's converter, with item 3's rule
+ * that -0.0 is a zero).  Per group g of four codes along k: keep the two of
+ * largest magnitude (ties to the lower index; -0.0 ranks as 0), emit the two
+ * source codes unchanged, lower index first, and the index nibble
+ * i0 | (i1 << 2).  Layout (version 1):
+ *   values: [n_pad, k/2] bytes, row-major, the kept codes group by group.
+ *   meta:   2048-byte tiles; tile (nt, kt) (nt < n_pad/128, kt < k/128) at
+ *           byte (nt*(k/128) + kt)*2048; inside, weight row 128*nt + r at
+ *           byte 16*r, byte b holding the nibble of group 32*kt + 2b in bits
+ *           0..3 and of group 32*kt + 2b + 1 in bits 4..7.
+ *   Rows n..n_pad-1: value 0x00 and nibble 0x4 everywhere.
+ *
+ *  w_q     device, [n, k] FP8 codes (w_dtype E4M3 or E5M2), row stride k,
+ *          16-byte aligned.  NaN codes are outside the contract.
+ *  values, meta  device, sizes above, 16-byte aligned.
+ */
+sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n,
+                             int64_t k, void* values, void* meta,
+                             void* stream);
+
+/*
+ * Inverse of sfp8_compress_24 (a checking aid): writes the dense [n, k]
+ * codes, 0x00 in dropped slots.  w_q 16-byte aligned, row stride k.
+ * An invalid nibble sets SFP8_DEVICE_CHECK_FAIL in the device status word.
+ */
+sfp8_status sfp8_decompress_24(const void* values, const void* meta,
+                               int64_t n, int64_t k, void* w_q, void* stream);
+
+/*
+ * Workspace for sfp8_sparse_linear on the current device (split-K partial
+ * sums and per-tile counters).  The counters part must be zero before the
+ * first call that uses a workspace; every call leaves it zero again (clear it
+ * again after a call that reported a device error).  sfp8_workspace_clear
+ * zeroes a workspace on a stream.
+ */
+size_t sfp8_sparse_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
+sfp8_status sfp8_workspace_clear(void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
+ * The sparse FP8 linear (item 1's operator; the four e4m3/e5m2 operand
+ * pairs of the page's per-dtype files are run-time choices here):
+ *     y[m, n] = bf16_RNE( acc[m, n] * s_a[m] * s_w[n] + bias[n] )
+ * with acc[m, n] = sum over kept slots of dec(A_q[m, k]) * dec(W_q[n, k]),
+ * accumulated in fp32 by the sm_100 sparse tensor cores.
+ *
+ *  a_q     device, [m, k] FP8 codes (a_dtype E4M3 or E5M2), row stride k,
+ *          16-byte aligned.
+ *  s_a     device, [m] float32.
+ *  values, meta  device, from sfp8_compress_24 for an [n, k] weight of
+ *          w_dtype (E4M3 or E5M2).
+ *  s_w     device, [n] float32.
+ *  bias    device, [n] bf16, or NULL for none.
+ *  y       device, [m, n] bf16, row stride n.
+ *  workspace  device, >= sfp8_sparse_linear_workspace_bytes(m, n, k) bytes,
+ *          16-byte aligned, counters zero (see above).
+ *  k % 128 == 0, k > 0; m, n >= 0.
+ */
+sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
+                               const float* s_a, int64_t m,
+                               const void* values, const void* meta,
+                               sfp8_dtype w_dtype, const float* s_w,
+                               int64_t n, int64_t k, const void* bias,
+                               void* y, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
+ * Reads (and with clear != 0, resets) the current device's status word.
+ * Synchronises the device first.  *flags receives SFP8_DEVICE_* bits.
+ * Returns SFP8_ERR_TIMEOUT / SFP8_ERR_DEVICE_CHECK when such a bit is set,
+ * SFP8_OK otherwise.
+ */
+sfp8_status sfp8_read_device_status(uint32_t* flags, int clear);
+
+const char* sfp8_status_string(sfp8_status s);
+int sfp8_layout_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFP8_H_ */

@@ -1,1 +1,25 @@
-"""Row-wise scaled 2:4 sparse FP8 linear for B200 (sm_100a)."""
+"""Row-wise scaled 2:4 sparse FP8 linear for B200 (sm_100a).
+
+The compute path is libsfp8.so (C ABI, include/sfp8.h); this package holds
+its build script, a ctypes binding with the same function names, a layer
+class on top of it, and the seeded synthetic-input generators.
+"""
+
+from .binding import (Sfp8Error, load_library, library_path, new_workspace,
+                      sfp8_quantize_rowwise, sfp8_prune_24, sfp8_padded_rows,
+                      sfp8_compressed_values_bytes, sfp8_compressed_meta_bytes,
+                      sfp8_compress_24, sfp8_decompress_24,
+                      sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
+                      sfp8_sparse_linear, sfp8_read_device_status,
+                      sfp8_status_string, sfp8_layout_version)
+from .layer import SparseFp8Linear
+
+__all__ = [
+    "Sfp8Error", "load_library", "library_path", "new_workspace",
+    "sfp8_quantize_rowwise", "sfp8_prune_24", "sfp8_padded_rows",
+    "sfp8_compressed_values_bytes", "sfp8_compressed_meta_bytes",
+    "sfp8_compress_24", "sfp8_decompress_24",
+    "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
+    "sfp8_sparse_linear", "sfp8_read_device_status", "sfp8_status_string",
+    "sfp8_layout_version", "SparseFp8Linear",
+]

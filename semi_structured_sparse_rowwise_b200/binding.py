@@ -1,0 +1,251 @@
+"""Thin Python binding of libsfp8.so (ctypes).
+
+Argument marshalling only: tensors are passed as raw device pointers with
+their sizes, on torch's current CUDA stream.  Every step of the layer runs in
+the library's CUDA kernels; there is no fallback of any kind.  If the library
+is missing or fails to load, every call raises.
+
+The functions carry the C names (``sfp8_quantize_rowwise`` and so on) and
+allocate their outputs with torch when none are given.
+"""
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+OK = 0
+STATUS_NAMES = {
+    0: "SFP8_OK", 1: "SFP8_ERR_INVALID_ARG", 2: "SFP8_ERR_UNSUPPORTED_SHAPE",
+    3: "SFP8_ERR_MISALIGNED", 4: "SFP8_ERR_UNSUPPORTED_DTYPE", 5: "SFP8_ERR_ARCH",
+    6: "SFP8_ERR_WORKSPACE", 7: "SFP8_ERR_CUDA", 8: "SFP8_ERR_TIMEOUT",
+    9: "SFP8_ERR_DEVICE_CHECK",
+}
+DTYPE = {"bf16": 0, "f16": 1, "f32": 2, "e4m3": 3, "e5m2": 4}
+TORCH_WIDE = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}
+DEVICE_TIMEOUT = 0x1
+DEVICE_CHECK_FAIL = 0x2
+
+# Every symbol declared in include/sfp8.h, with its C signature.
+_c_void_p, _i64, _sz, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+SIGNATURES = {
+    "sfp8_quantize_rowwise": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _i32,
+                                     _c_void_p, _c_void_p]),
+    "sfp8_prune_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _c_void_p]),
+    "sfp8_padded_rows": (_i64, [_i64]),
+    "sfp8_compressed_values_bytes": (_sz, [_i64, _i64]),
+    "sfp8_compressed_meta_bytes": (_sz, [_i64, _i64]),
+    "sfp8_compress_24": (_i32, [_c_void_p, _i32, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "sfp8_decompress_24": (_i32, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "sfp8_sparse_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "sfp8_workspace_clear": (_i32, [_c_void_p, _sz, _c_void_p]),
+    "sfp8_sparse_linear": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _c_void_p, _i32,
+                                  _c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _sz,
+                                  _c_void_p]),
+    "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
+    "sfp8_status_string": (ctypes.c_char_p, [_i32]),
+    "sfp8_layout_version": (_i32, []),
+}
+
+_LIB = None
+
+
+class Sfp8Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (what, STATUS_NAMES.get(status, "?"), status))
+
+
+def library_path():
+    return _build.LIB_PATH
+
+
+def load_library():
+    """Loads libsfp8.so from the package directory (raises if absent)."""
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(
+                "libsfp8.so is not built (%s); run "
+                "`python -m semi_structured_sparse_rowwise_b200.build`" % path)
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = lib
+    return _LIB
+
+
+def _check(status, what):
+    if status != OK:
+        raise Sfp8Error(status, what)
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _fp8_name(d):
+    if d not in ("e4m3", "e5m2"):
+        raise ValueError("fp8 dtype must be 'e4m3' or 'e5m2'")
+    return d
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors")
+
+
+def sfp8_quantize_rowwise(x, q_dtype="e4m3", q=None, scales=None):
+    """x [rows, cols] bf16/f16/f32 (unit column stride) -> (q uint8, scales f32)."""
+    lib = load_library()
+    _require_cuda(x)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    rows, cols = x.shape
+    xd = TORCH_WIDE.get(x.dtype)
+    if xd is None:
+        raise ValueError("x dtype must be bfloat16, float16 or float32")
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((rows,), dtype=torch.float32, device=x.device)
+    ld = x.stride(0) if rows > 1 else cols
+    with torch.cuda.device(x.device):
+        st = lib.sfp8_quantize_rowwise(_ptr(x), DTYPE[xd], rows, cols, ld, _ptr(q),
+                                       DTYPE[_fp8_name(q_dtype)], _ptr(scales), _stream(x.device))
+    _check(st, "sfp8_quantize_rowwise")
+    return q, scales
+
+
+def sfp8_prune_24(w, out=None):
+    """2:4 magnitude prune along rows; w [rows, cols] bf16/f16/f32."""
+    lib = load_library()
+    _require_cuda(w)
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be 2-D with unit column stride")
+    wd = TORCH_WIDE.get(w.dtype)
+    if wd is None:
+        raise ValueError("w dtype must be bfloat16, float16 or float32")
+    rows, cols = w.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=w.dtype, device=w.device)
+    ld = w.stride(0) if rows > 1 else cols
+    with torch.cuda.device(w.device):
+        st = lib.sfp8_prune_24(_ptr(w), DTYPE[wd], rows, cols, ld, _ptr(out), _stream(w.device))
+    _check(st, "sfp8_prune_24")
+    return out
+
+
+def sfp8_padded_rows(n):
+    return int(load_library().sfp8_padded_rows(n))
+
+
+def sfp8_compressed_values_bytes(n, k):
+    return int(load_library().sfp8_compressed_values_bytes(n, k))
+
+
+def sfp8_compressed_meta_bytes(n, k):
+    return int(load_library().sfp8_compressed_meta_bytes(n, k))
+
+
+def sfp8_compress_24(w_q, w_dtype="e4m3", values=None, meta=None):
+    """w_q [n, k] uint8 FP8 codes -> (values, meta) in the library's layout."""
+    lib = load_library()
+    _require_cuda(w_q)
+    if w_q.dim() != 2 or not w_q.is_contiguous() or w_q.dtype != torch.uint8:
+        raise ValueError("w_q must be a contiguous 2-D uint8 tensor")
+    n, k = w_q.shape
+    if values is None:
+        values = torch.empty((lib.sfp8_compressed_values_bytes(n, k),), dtype=torch.uint8,
+                             device=w_q.device)
+    if meta is None:
+        meta = torch.empty((lib.sfp8_compressed_meta_bytes(n, k),), dtype=torch.uint8,
+                           device=w_q.device)
+    with torch.cuda.device(w_q.device):
+        st = lib.sfp8_compress_24(_ptr(w_q), DTYPE[_fp8_name(w_dtype)], n, k, _ptr(values),
+                                  _ptr(meta), _stream(w_q.device))
+    _check(st, "sfp8_compress_24")
+    return values, meta
+
+
+def sfp8_decompress_24(values, meta, n, k, out=None):
+    lib = load_library()
+    _require_cuda(values, meta)
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.uint8, device=values.device)
+    with torch.cuda.device(values.device):
+        st = lib.sfp8_decompress_24(_ptr(values), _ptr(meta), n, k, _ptr(out),
+                                    _stream(values.device))
+    _check(st, "sfp8_decompress_24")
+    return out
+
+
+def sfp8_sparse_linear_workspace_bytes(m, n, k, device=None):
+    lib = load_library()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(lib.sfp8_sparse_linear_workspace_bytes(m, n, k))
+
+
+def new_workspace(m, n, k, device):
+    """A zeroed workspace for sfp8_sparse_linear(m, n, k) on `device`."""
+    nbytes = sfp8_sparse_linear_workspace_bytes(m, n, k, device)
+    return torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=device)
+
+
+def sfp8_workspace_clear(workspace):
+    lib = load_library()
+    with torch.cuda.device(workspace.device):
+        st = lib.sfp8_workspace_clear(_ptr(workspace), workspace.numel(),
+                                      _stream(workspace.device))
+    _check(st, "sfp8_workspace_clear")
+
+
+def sfp8_sparse_linear(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k, bias=None,
+                       out=None, workspace=None):
+    """y [m, n] bf16 = (s_a s_w^T) * (A_q . W_q^T) + bias."""
+    lib = load_library()
+    _require_cuda(a_q, s_a, values, meta, s_w, bias)
+    if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
+        raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
+    m = a_q.shape[0]
+    if a_q.shape[1] != k:
+        raise ValueError("a_q has %d columns, expected k=%d" % (a_q.shape[1], k))
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
+    if workspace is None:
+        workspace = new_workspace(m, n, k, a_q.device)
+    if bias is not None and bias.dtype != torch.bfloat16:
+        raise ValueError("bias must be bfloat16")
+    with torch.cuda.device(a_q.device):
+        st = lib.sfp8_sparse_linear(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
+                                    _ptr(values), _ptr(meta), DTYPE[_fp8_name(w_dtype)],
+                                    _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
+                                    workspace.numel(), _stream(a_q.device))
+    _check(st, "sfp8_sparse_linear")
+    return out
+
+
+def sfp8_read_device_status(clear=True):
+    """(status, flags) of the current device's status word; synchronises."""
+    lib = load_library()
+    flags = ctypes.c_uint32(0)
+    st = lib.sfp8_read_device_status(ctypes.byref(flags), 1 if clear else 0)
+    return st, flags.value
+
+
+def sfp8_status_string(status):
+    return load_library().sfp8_status_string(status).decode()
+
+
+def sfp8_layout_version():
+    return int(load_library().sfp8_layout_version())

@@ -1,0 +1,456 @@
+// C-ABI entry points of libsfp8.so (declared in include/sfp8.h): argument
+// validation, tile planning, TMA descriptor encoding and kernel launches.
+// The kernels are in the .cuh files included below; this is the only
+// translation unit of the library.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sfp8.h"
+#include "device_common.cuh"
+#include "quantize_rowwise.cuh"
+#include "sparse24_pack.cuh"
+#include "sparse_linear.cuh"
+
+namespace sfp8 {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool is_sm100 = false;
+  int num_sms = 0;
+  bool smem_attr_set[8] = {};
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+sfp8_status current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SFP8_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SFP8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& d = g_devices[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SFP8_ERR_CUDA;
+    d.is_sm100 = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    d.probed = true;
+  }
+  if (!d.is_sm100) return SFP8_ERR_ARCH;
+  *out = &d;
+  return SFP8_OK;
+}
+
+sfp8_status get_encoder(EncodeTiledFn* fn) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_encode == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr)
+      return SFP8_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = g_encode;
+  return SFP8_OK;
+}
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline sfp8_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SFP8_OK : SFP8_ERR_CUDA;
+}
+
+inline int elem_size(sfp8_dtype t) {
+  switch (t) {
+    case SFP8_BF16:
+    case SFP8_F16:
+      return 2;
+    case SFP8_F32:
+      return 4;
+    case SFP8_E4M3:
+    case SFP8_E5M2:
+      return 1;
+  }
+  return 0;
+}
+
+inline bool is_fp8(sfp8_dtype t) { return t == SFP8_E4M3 || t == SFP8_E5M2; }
+inline bool is_wide(sfp8_dtype t) { return t == SFP8_BF16 || t == SFP8_F16 || t == SFP8_F32; }
+
+// ------------------------------------------------------------------ quantise
+
+template <typename T, int kFmt>
+sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
+                            float* scales, cudaStream_t st) {
+  const T* xp = static_cast<const T*>(x);
+  uint8_t* qp = static_cast<uint8_t*>(q);
+  if (cols == 0) {
+    const int64_t blocks = (rows + 255) / 256;
+    quantize_empty_rows_kernel<kFmt><<<static_cast<unsigned>(blocks), 256, 0, st>>>(rows, scales);
+    return launch_status();
+  }
+  constexpr int P = InputTraits<T>::kPerVec;
+  const int64_t nvec = cols / P;
+  constexpr int kChunks = 8;
+  if (nvec <= 32 * kChunks) {
+    const int64_t blocks = (rows + 7) / 8;
+    quantize_rowwise_kernel<T, kFmt, 32, kChunks>
+        <<<static_cast<unsigned>(blocks), 256, 0, st>>>(xp, rows, cols, ld, qp, scales);
+  } else if (nvec <= 128 * kChunks) {
+    const int64_t blocks = (rows + 1) / 2;
+    quantize_rowwise_kernel<T, kFmt, 128, kChunks>
+        <<<static_cast<unsigned>(blocks), 256, 0, st>>>(xp, rows, cols, ld, qp, scales);
+  } else if (nvec <= 512 * kChunks) {
+    quantize_rowwise_kernel<T, kFmt, 512, kChunks>
+        <<<static_cast<unsigned>(rows), 512, 0, st>>>(xp, rows, cols, ld, qp, scales);
+  } else {
+    quantize_rowwise_long_kernel<T, kFmt>
+        <<<static_cast<unsigned>(rows), 1024, 0, st>>>(xp, rows, cols, ld, qp, scales);
+  }
+  return launch_status();
+}
+
+template <typename T>
+sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
+                                sfp8_dtype q_dtype, float* scales, cudaStream_t st) {
+  if (q_dtype == SFP8_E4M3) return launch_quantize<T, SFP8_E4M3>(x, rows, cols, ld, q, scales, st);
+  return launch_quantize<T, SFP8_E5M2>(x, rows, cols, ld, q, scales, st);
+}
+
+// ------------------------------------------------------------------ linear plan
+
+struct LinearPlan {
+  int bn;
+  int grid;
+  int m_tiles;
+  int k_steps;
+  long long n_tiles;
+  long long tiles;
+  long long iters;
+  size_t partial_bytes;
+  size_t counter_bytes;
+};
+
+int choose_bn(int64_t m) {
+  if (m <= 16) return 16;
+  if (m <= 32) return 32;
+  if (m <= 64) return 64;
+  if (m <= 128) return 128;
+  return 128;
+}
+
+LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
+  LinearPlan pl{};
+  pl.bn = choose_bn(m);
+  pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
+  pl.k_steps = static_cast<int>(k / kStepK);
+  pl.n_tiles = (n + kTileN - 1) / kTileN;
+  pl.tiles = pl.n_tiles * pl.m_tiles;
+  pl.iters = pl.tiles * pl.k_steps;
+  pl.grid = static_cast<int>(pl.iters < num_sms ? pl.iters : num_sms);
+  if (pl.grid < 1) pl.grid = 1;
+  pl.partial_bytes = static_cast<size_t>(pl.grid) * 2 * pl.bn * kTileN * sizeof(float);
+  pl.partial_bytes = (pl.partial_bytes + 255) & ~static_cast<size_t>(255);
+  pl.counter_bytes = static_cast<size_t>(pl.tiles) * 4 * sizeof(unsigned int);
+  return pl;
+}
+
+template <int BN>
+sfp8_status launch_linear_bn(DeviceInfo* dev, int slot, const CUtensorMap& tw,
+                             const CUtensorMap& ta, const LinearParams& prm, cudaStream_t st) {
+  using Cfg = LinearCfg<BN>;
+  auto kern = sparse_linear_kernel<BN>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!dev->smem_attr_set[slot]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cfg::kSmemBytes) != cudaSuccess)
+        return SFP8_ERR_CUDA;
+      dev->smem_attr_set[slot] = true;
+    }
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(prm.grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tw, ta, prm) != cudaSuccess) {
+    cudaGetLastError();
+    return SFP8_ERR_CUDA;
+  }
+  return SFP8_OK;
+}
+
+sfp8_status encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                         uint64_t row_stride, uint32_t box_inner, uint32_t box_outer,
+                         CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = nullptr;
+  sfp8_status s = get_encoder(&enc);
+  if (s != SFP8_OK) return s;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sfp8
+
+using namespace sfp8;
+
+extern "C" {
+
+const char* sfp8_status_string(sfp8_status s) {
+  switch (s) {
+    case SFP8_OK: return "ok";
+    case SFP8_ERR_INVALID_ARG: return "invalid argument";
+    case SFP8_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case SFP8_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case SFP8_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case SFP8_ERR_ARCH: return "current device is not sm_100";
+    case SFP8_ERR_WORKSPACE: return "workspace missing or too small";
+    case SFP8_ERR_CUDA: return "CUDA error";
+    case SFP8_ERR_TIMEOUT: return "device-side wait timed out";
+    case SFP8_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int sfp8_layout_version(void) { return SFP8_LAYOUT_VERSION; }
+
+int64_t sfp8_padded_rows(int64_t n) {
+  if (n < 0) return -1;
+  return ((n + kTileN - 1) / kTileN) * kTileN;
+}
+
+size_t sfp8_compressed_values_bytes(int64_t n, int64_t k) {
+  if (n < 0 || k < 0) return 0;
+  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k / 2);
+}
+
+size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k) {
+  if (n < 0 || k < 0) return 0;
+  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k / 8);
+}
+
+sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype, int64_t rows, int64_t cols,
+                                  int64_t ld_x, void* q, sfp8_dtype q_dtype, float* scales,
+                                  void* stream) {
+  if (!is_wide(x_dtype) || !is_fp8(q_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (rows < 0 || cols < 0 || ld_x < cols) return SFP8_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (rows >= (int64_t(1) << 31) / 8) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return SFP8_OK;
+  if (scales == nullptr || (cols > 0 && (x == nullptr || q == nullptr)))
+    return SFP8_ERR_INVALID_ARG;
+  const int es = elem_size(x_dtype);
+  if (cols > 0 && (!aligned(x, 16) || !aligned(q, 16) || (ld_x * es) % 16 != 0))
+    return SFP8_ERR_MISALIGNED;
+  if (!aligned(scales, 4)) return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (x_dtype) {
+    case SFP8_BF16:
+      return launch_quantize_fmt<__nv_bfloat16>(x, rows, cols, ld_x, q, q_dtype, scales, st);
+    case SFP8_F16:
+      return launch_quantize_fmt<__half>(x, rows, cols, ld_x, q, q_dtype, scales, st);
+    default:
+      return launch_quantize_fmt<float>(x, rows, cols, ld_x, q, q_dtype, scales, st);
+  }
+}
+
+sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows, int64_t cols,
+                          int64_t ld, void* out, void* stream) {
+  if (!is_wide(dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (rows < 0 || cols < 0 || ld < cols) return SFP8_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0 || cols == 0) return SFP8_OK;
+  if (w == nullptr || out == nullptr) return SFP8_ERR_INVALID_ARG;
+  const int es = elem_size(dtype);
+  if (!aligned(w, 16) || !aligned(out, 16) || (ld * es) % 16 != 0) return SFP8_ERR_MISALIGNED;
+  if (w == out && ld != cols) return SFP8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t vecs = rows * (cols * es / 16);
+  int64_t blocks = (vecs + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(dev->num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  if (es == 2) {
+    prune24_kernel<uint16_t><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint16_t*>(w), rows, cols, ld, static_cast<uint16_t*>(out));
+  } else {
+    prune24_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        static_cast<const uint32_t*>(w), rows, cols, ld, static_cast<uint32_t*>(out));
+  }
+  return launch_status();
+}
+
+sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n, int64_t k,
+                             void* values, void* meta, void* stream) {
+  if (!is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
+  if (k % kStepK != 0 || k == 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return SFP8_OK;
+  if (k / kStepK > 65535 || sfp8_padded_rows(n) / kTileN > 65535) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (w_q == nullptr || values == nullptr || meta == nullptr) return SFP8_ERR_INVALID_ARG;
+  if (!aligned(w_q, 16) || !aligned(values, 16) || !aligned(meta, 16)) return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  dim3 grid(static_cast<unsigned>(k / kStepK), static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
+  compress24_kernel<<<grid, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(w_q), n, k, static_cast<uint8_t*>(values),
+      static_cast<uint8_t*>(meta));
+  return launch_status();
+}
+
+sfp8_status sfp8_decompress_24(const void* values, const void* meta, int64_t n, int64_t k,
+                               void* w_q, void* stream) {
+  if (n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
+  if (k % kStepK != 0 || k == 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return SFP8_OK;
+  if (k / kStepK > 65535 || sfp8_padded_rows(n) / kTileN > 65535) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (w_q == nullptr || values == nullptr || meta == nullptr) return SFP8_ERR_INVALID_ARG;
+  if (!aligned(w_q, 16) || !aligned(values, 16) || !aligned(meta, 16)) return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  dim3 grid(static_cast<unsigned>(k / kStepK), static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
+  decompress24_kernel<<<grid, 512, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(values), static_cast<const uint8_t*>(meta), n, k,
+      static_cast<uint8_t*>(w_q));
+  return launch_status();
+}
+
+size_t sfp8_sparse_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % kStepK != 0) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const LinearPlan pl = make_plan(m, n, k, sms);
+  return pl.partial_bytes + pl.counter_bytes;
+}
+
+sfp8_status sfp8_workspace_clear(void* workspace, size_t workspace_bytes, void* stream) {
+  if (workspace_bytes == 0) return SFP8_OK;
+  if (workspace == nullptr) return SFP8_ERR_INVALID_ARG;
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SFP8_OK
+             : SFP8_ERR_CUDA;
+}
+
+sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_a, int64_t m,
+                               const void* values, const void* meta, sfp8_dtype w_dtype,
+                               const float* s_w, int64_t n, int64_t k, const void* bias, void* y,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
+  if (k == 0 || k % kStepK != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 31))
+    return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m == 0 || n == 0) return SFP8_OK;
+  if (a_q == nullptr || s_a == nullptr || values == nullptr || meta == nullptr ||
+      s_w == nullptr || y == nullptr)
+    return SFP8_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(values, 16) || !aligned(meta, 16) || !aligned(s_a, 4) ||
+      !aligned(s_w, 4) || !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
+    return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  const LinearPlan pl = make_plan(m, n, k, dev->num_sms);
+  if (workspace == nullptr || workspace_bytes < pl.partial_bytes + pl.counter_bytes)
+    return SFP8_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+
+  CUtensorMap tw, ta;
+  const int64_t n_pad = sfp8_padded_rows(n);
+  s = encode_2d_u8(&tw, values, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n_pad),
+                   static_cast<uint64_t>(k / 2), kStepK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != SFP8_OK) return s;
+  s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
+                   static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SFP8_OK) return s;
+
+  LinearParams prm{};
+  prm.meta = static_cast<const uint8_t*>(meta);
+  prm.s_a = s_a;
+  prm.s_w = s_w;
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.y = static_cast<__nv_bfloat16*>(y);
+  prm.partials = static_cast<float*>(workspace);
+  prm.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes);
+  prm.m = static_cast<int>(m);
+  prm.n = static_cast<int>(n);
+  prm.k = static_cast<int>(k);
+  prm.m_tiles = pl.m_tiles;
+  prm.k_steps = pl.k_steps;
+  prm.tiles = pl.tiles;
+  prm.iters = pl.iters;
+  prm.grid = pl.grid;
+  // MMA A operand = weight, B operand = activation.
+  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
+                                kTileN, static_cast<uint32_t>(pl.bn), true);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (pl.bn) {
+    case 16: return launch_linear_bn<16>(dev, 0, tw, ta, prm, st);
+    case 32: return launch_linear_bn<32>(dev, 1, tw, ta, prm, st);
+    case 64: return launch_linear_bn<64>(dev, 2, tw, ta, prm, st);
+    case 128: return launch_linear_bn<128>(dev, 3, tw, ta, prm, st);
+    default: return launch_linear_bn<256>(dev, 4, tw, ta, prm, st);
+  }
+}
+
+sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
+  if (flags == nullptr) return SFP8_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SFP8_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return SFP8_ERR_CUDA;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+      return SFP8_ERR_CUDA;
+  }
+  *flags = v;
+  if (v & SFP8_DEVICE_TIMEOUT) return SFP8_ERR_TIMEOUT;
+  if (v & SFP8_DEVICE_CHECK_FAIL) return SFP8_ERR_DEVICE_CHECK;
+  return SFP8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,165 @@
+// 2:4 pruning, compression and decompression kernels.
+//
+// Page "Add CUTLASS-based row-wise scaled sparse FP8 kernel" (pytorch/ao pull
+// request 1671): item 1's converter of FP8 data to the compressed 2:4 format,
+// with item 3's rule that -0.0 counts as zero.  The selection is integer-only:
+// for finite FP8 codes (and finite bf16/fp16/fp32 bit patterns) the value of
+// `bits & ~sign` grows with |value|, and -0.0 has magnitude bits 0.
+//
+// In a group with magnitudes m0..m3, element j is kept iff fewer than two
+// elements beat it, where i beats j when m_i > m_j, or m_i == m_j and i < j
+// (ties to the lower index).
+//
+// Compressed layout (version 1), for an [n, k] weight, n_pad = ceil(n/128)*128:
+//   values [n_pad, k/2] row-major, kept codes group by group (lower index
+//   first); meta in 2048-byte tiles, tile (nt, kt) at (nt*(k/128)+kt)*2048,
+//   row r of the tile at 16*r, byte b = nibbles of groups 2b (bits 0..3) and
+//   2b+1 (bits 4..7) of that 128-wide k tile.  Padding rows: 0x00 values,
+//   nibble 0x4.  Each tile is exactly the 128-lane x 128-bit block that the
+//   GEMM copies into tensor memory for one 128-wide k step of 128 weight rows.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace sfp8 {
+
+// Keep mask (bit j set = element j kept) from four magnitudes.
+__device__ __forceinline__ uint32_t keep_mask4(uint32_t m0, uint32_t m1, uint32_t m2,
+                                               uint32_t m3) {
+  // beats[i][j]: i beats j
+  const uint32_t b01 = m0 >= m1, b02 = m0 >= m2, b03 = m0 >= m3;  // i < j: ties to i
+  const uint32_t b12 = m1 >= m2, b13 = m1 >= m3, b23 = m2 >= m3;
+  // number of elements beating j
+  const uint32_t r0 = (1 - b01) + (1 - b02) + (1 - b03);
+  const uint32_t r1 = b01 + (1 - b12) + (1 - b13);
+  const uint32_t r2 = b02 + b12 + (1 - b23);
+  const uint32_t r3 = b03 + b13 + b23;
+  return (r0 < 2 ? 1u : 0u) | (r1 < 2 ? 2u : 0u) | (r2 < 2 ? 4u : 0u) | (r3 < 2 ? 8u : 0u);
+}
+
+// Kept indices i0 < i1 from a 4-bit mask with exactly two bits set.
+__device__ __forceinline__ void kept_indices(uint32_t mask, uint32_t& i0, uint32_t& i1) {
+  i0 = __ffs(mask) - 1;
+  i1 = __ffs(mask & (mask - 1)) - 1;
+}
+
+// ---------------------------------------------------------------- prune
+
+template <typename Bits>
+struct PruneTraits;
+template <>
+struct PruneTraits<uint16_t> {
+  static constexpr uint32_t kMag = 0x7FFFu;
+};
+template <>
+struct PruneTraits<uint32_t> {
+  static constexpr uint32_t kMag = 0x7FFFFFFFu;
+};
+
+// One 16-byte vector per thread: 2 groups of 16-bit elements or 1 group of
+// 32-bit elements.  Dropped elements become +0.0 (all bits zero).
+template <typename Bits>
+__global__ void prune24_kernel(const Bits* __restrict__ w, int64_t rows, int64_t cols,
+                               int64_t ld, Bits* __restrict__ out) {
+  constexpr int kPer = 16 / sizeof(Bits);
+  const int64_t vec_per_row = cols / kPer;
+  const int64_t total = rows * vec_per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / vec_per_row;
+    const int64_t c = (i % vec_per_row) * kPer;
+    uint4 v = *reinterpret_cast<const uint4*>(w + r * ld + c);
+    Bits e[kPer];
+    *reinterpret_cast<uint4*>(e) = v;
+#pragma unroll
+    for (int g = 0; g < kPer / 4; ++g) {
+      const uint32_t M = PruneTraits<Bits>::kMag;
+      const uint32_t keep = keep_mask4(e[4 * g] & M, e[4 * g + 1] & M, e[4 * g + 2] & M,
+                                       e[4 * g + 3] & M);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (!((keep >> j) & 1)) e[4 * g + j] = 0;
+    }
+    *reinterpret_cast<uint4*>(out + r * cols + c) = *reinterpret_cast<uint4*>(e);
+  }
+}
+
+// ---------------------------------------------------------------- compress
+
+// Block = 512 threads = 128 rows x 4 threads; blockIdx.x = k tile, blockIdx.y
+// = row tile.  Each thread turns 32 input codes (8 groups) into 16 value
+// bytes and 4 metadata bytes.
+__global__ void __launch_bounds__(512)
+    compress24_kernel(const uint8_t* __restrict__ wq, int64_t n, int64_t k,
+                      uint8_t* __restrict__ values, uint8_t* __restrict__ meta) {
+  const int r = threadIdx.x / 4;   // row inside the tile
+  const int j = threadIdx.x % 4;   // 32-code chunk inside the 128-wide k tile
+  const int64_t kt = blockIdx.x;
+  const int64_t nt = blockIdx.y;
+  const int64_t row = nt * 128 + r;
+  const int64_t ktiles = k / 128;
+  uint32_t vout[4];
+  uint32_t mout = 0;
+  if (row < n) {
+    const uint8_t* src = wq + row * k + kt * 128 + 32 * j;
+    uint32_t in[8];
+    *reinterpret_cast<uint4*>(&in[0]) = __ldg(reinterpret_cast<const uint4*>(src));
+    *reinterpret_cast<uint4*>(&in[4]) = __ldg(reinterpret_cast<const uint4*>(src + 16));
+    uint32_t vb[16];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const uint32_t word = in[g];   // codes 4g..4g+3 of this chunk, little-endian
+      const uint32_t c0 = word & 0xFF, c1 = (word >> 8) & 0xFF, c2 = (word >> 16) & 0xFF,
+                     c3 = word >> 24;
+      const uint32_t keep = keep_mask4(c0 & 0x7F, c1 & 0x7F, c2 & 0x7F, c3 & 0x7F);
+      uint32_t i0, i1;
+      kept_indices(keep, i0, i1);
+      vb[2 * g] = (word >> (8 * i0)) & 0xFF;
+      vb[2 * g + 1] = (word >> (8 * i1)) & 0xFF;
+      mout |= (i0 | (i1 << 2)) << (4 * g);
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      vout[w] = vb[4 * w] | (vb[4 * w + 1] << 8) | (vb[4 * w + 2] << 16) | (vb[4 * w + 3] << 24);
+  } else {
+    vout[0] = vout[1] = vout[2] = vout[3] = 0;
+    mout = 0x44444444u;   // indices (0, 1) in every group
+  }
+  *reinterpret_cast<uint4*>(values + row * (k / 2) + kt * 64 + 16 * j) =
+      make_uint4(vout[0], vout[1], vout[2], vout[3]);
+  *reinterpret_cast<uint32_t*>(meta + (nt * ktiles + kt) * 2048 + 16 * r + 4 * j) = mout;
+}
+
+// Inverse: same thread mapping, n real rows only.
+__global__ void __launch_bounds__(512)
+    decompress24_kernel(const uint8_t* __restrict__ values, const uint8_t* __restrict__ meta,
+                        int64_t n, int64_t k, uint8_t* __restrict__ wq) {
+  const int r = threadIdx.x / 4;
+  const int j = threadIdx.x % 4;
+  const int64_t kt = blockIdx.x;
+  const int64_t nt = blockIdx.y;
+  const int64_t row = nt * 128 + r;
+  if (row >= n) return;
+  const int64_t ktiles = k / 128;
+  const uint4 vv = *reinterpret_cast<const uint4*>(values + row * (k / 2) + kt * 64 + 16 * j);
+  const uint32_t mm =
+      *reinterpret_cast<const uint32_t*>(meta + (nt * ktiles + kt) * 2048 + 16 * r + 4 * j);
+  const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+  uint32_t out[8];
+  bool bad = false;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const uint32_t nib = (mm >> (4 * g)) & 0xF;
+    const uint32_t i0 = nib & 3, i1 = nib >> 2;
+    if (i0 >= i1) bad = true;
+    const uint32_t v0 = (vw[g / 2] >> (16 * (g % 2))) & 0xFF;
+    const uint32_t v1 = (vw[g / 2] >> (16 * (g % 2) + 8)) & 0xFF;
+    out[g] = (v0 << (8 * i0)) | (i1 > i0 ? (v1 << (8 * i1)) : 0);
+  }
+  if (bad) report_device_error(SFP8_DEVICE_CHECK_FAIL);
+  uint8_t* dst = wq + row * k + kt * 128 + 32 * j;
+  *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+  *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+}  // namespace sfp8

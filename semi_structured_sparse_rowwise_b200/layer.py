@@ -1,0 +1,68 @@
+"""The layer a user calls: a prepared 2:4 sparse FP8 weight and its forward.
+
+Weight preparation (once, as the page "Add CUTLASS-based row-wise scaled
+sparse FP8 kernel", pytorch/ao pull request 1671, does at ``quantize_()`` time,
+its items 1, 3 and 4): 2:4 magnitude prune -> row-wise FP8 quantisation ->
+2:4 compression.  Forward (per call): dynamic row-wise FP8 quantisation of the
+activation -> sparse FP8 GEMM with the scale/bias epilogue.  Every step is a
+kernel of libsfp8.so; torch only provides memory and streams.
+"""
+
+import torch
+
+from . import binding as B
+
+
+class SparseFp8Linear:
+    """y = (s_a s_w^T) * (A_q W_q^T) + bias with a 2:4 compressed FP8 weight."""
+
+    def __init__(self, weight, bias=None, w_dtype="e4m3", a_dtype="e4m3", prune=True):
+        if weight.dim() != 2:
+            raise ValueError("weight must be [out_features, in_features]")
+        self.n, self.k = weight.shape
+        self.w_dtype = w_dtype
+        self.a_dtype = a_dtype
+        self.device = weight.device
+        w = B.sfp8_prune_24(weight.contiguous()) if prune else weight.contiguous()
+        w_q, self.s_w = B.sfp8_quantize_rowwise(w, w_dtype)
+        self.values, self.meta = B.sfp8_compress_24(w_q, w_dtype)
+        self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
+        self._ws = {}
+
+    @classmethod
+    def from_compressed(cls, values, meta, s_w, n, k, bias=None, w_dtype="e4m3",
+                        a_dtype="e4m3"):
+        """A layer over an already compressed weight (values, meta, s_w)."""
+        self = cls.__new__(cls)
+        self.n, self.k = n, k
+        self.w_dtype, self.a_dtype = w_dtype, a_dtype
+        self.device = values.device
+        self.values, self.meta, self.s_w = values, meta, s_w
+        self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
+        self._ws = {}
+        return self
+
+    def workspace(self, m):
+        ws = self._ws.get(m)
+        if ws is None:
+            ws = B.new_workspace(m, self.n, self.k, self.device)
+            self._ws[m] = ws
+        return ws
+
+    def forward(self, x, out=None):
+        """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16."""
+        a_q, s_a = B.sfp8_quantize_rowwise(x, self.a_dtype)
+        return B.sfp8_sparse_linear(a_q, self.a_dtype, s_a, self.values, self.meta,
+                                    self.w_dtype, self.s_w, self.n, self.k, bias=self.bias,
+                                    out=out, workspace=self.workspace(x.shape[0]))
+
+    __call__ = forward
+
+    def forward_host(self, x_host, y_host, x_dev=None, y_dev=None):
+        """Host-buffer forward: x_host (pinned) -> device -> layer -> y_host."""
+        if x_dev is None:
+            x_dev = torch.empty(x_host.shape, dtype=x_host.dtype, device=self.device)
+        x_dev.copy_(x_host, non_blocking=True)
+        y = self.forward(x_dev, out=y_dev)
+        y_host.copy_(y, non_blocking=True)
+        return y_host

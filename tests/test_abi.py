@@ -1,0 +1,112 @@
+"""The C-ABI library builds, loads and exports every symbol that
+include/sfp8.h declares; host-side validation answers without a GPU.
+
+None of these tests launches a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from semi_structured_sparse_rowwise_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sfp8.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sfp8_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("sfp8_quantize_rowwise", "sfp8_compress_24", "sfp8_sparse_linear"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(binding.SIGNATURES), (set(names) ^ set(binding.SIGNATURES))
+
+
+def test_layout_constants_match(lib):
+    assert lib.sfp8_layout_version() == 1 == oracle.layout.LAYOUT_VERSION
+    for n in (0, 1, 127, 128, 129, 14336, 28672):
+        assert lib.sfp8_padded_rows(n) == oracle.padded_rows(n)
+        for k in (128, 4096, 14336):
+            assert lib.sfp8_compressed_values_bytes(n, k) == oracle.values_bytes(n, k)
+            assert lib.sfp8_compressed_meta_bytes(n, k) == oracle.meta_bytes(n, k)
+
+
+def test_status_strings(lib):
+    for code in range(10):
+        s = lib.sfp8_status_string(code)
+        assert s and s != b"unknown status"
+    assert lib.sfp8_status_string(99) == b"unknown status"
+
+
+FAKE = ctypes.c_void_p(0x10000)        # never dereferenced: rejected before use
+FAKE_ODD = ctypes.c_void_p(0x10001)
+
+
+def test_quantize_validation_without_gpu(lib):
+    q = lib.sfp8_quantize_rowwise
+    assert q(FAKE, 9, 4, 16, 16, FAKE, 3, FAKE, None) == 4       # bad input dtype
+    assert q(FAKE, 0, 4, 16, 16, FAKE, 0, FAKE, None) == 4       # bf16 output
+    assert q(FAKE, 0, -1, 16, 16, FAKE, 3, FAKE, None) == 1      # negative rows
+    assert q(FAKE, 0, 4, 16, 8, FAKE, 3, FAKE, None) == 1        # ld < cols
+    assert q(FAKE, 0, 4, 24, 24, FAKE, 3, FAKE, None) == 2       # cols % 16
+    assert q(FAKE, 0, 0, 16, 16, FAKE, 3, FAKE, None) == 0       # empty: no-op
+    assert q(None, 0, 4, 16, 16, FAKE, 3, FAKE, None) == 1       # null x
+    assert q(FAKE_ODD, 0, 4, 16, 16, FAKE, 3, FAKE, None) == 3   # misaligned x
+    assert q(FAKE, 0, 4, 16, 20, FAKE, 3, FAKE, None) == 3       # ld*2 % 16
+
+
+def test_prune_compress_validation_without_gpu(lib):
+    assert lib.sfp8_prune_24(FAKE, 3, 4, 16, 16, FAKE, None) == 4
+    assert lib.sfp8_prune_24(FAKE, 0, 4, 20, 20, FAKE, None) == 2
+    assert lib.sfp8_prune_24(FAKE, 0, 4, 16, 32, FAKE, None) == 1   # in place needs ld == cols
+    assert lib.sfp8_compress_24(FAKE, 0, 4, 128, FAKE, FAKE, None) == 4
+    assert lib.sfp8_compress_24(FAKE, 3, 4, 192, FAKE, FAKE, None) == 2
+    assert lib.sfp8_compress_24(FAKE, 3, 4, 0, FAKE, FAKE, None) == 2
+    assert lib.sfp8_compress_24(FAKE, 3, 0, 128, FAKE, FAKE, None) == 0
+    assert lib.sfp8_compress_24(FAKE_ODD, 3, 4, 128, FAKE, FAKE, None) == 3
+    assert lib.sfp8_decompress_24(FAKE, FAKE, 4, 100, FAKE, None) == 2
+
+
+def test_linear_validation_without_gpu(lib):
+    f = lib.sfp8_sparse_linear
+    args = [FAKE, 3, FAKE, 16, FAKE, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE, 1 << 20, None]
+
+    def call(**kw):
+        a = list(args)
+        names = ["a_q", "a_dt", "s_a", "m", "vals", "meta", "w_dt", "s_w", "n", "k", "bias",
+                 "y", "ws", "wsb", "stream"]
+        for key, v in kw.items():
+            a[names.index(key)] = v
+        return f(*a)
+    assert call(a_dt=0) == 4
+    assert call(w_dt=2) == 4
+    assert call(k=0) == 2
+    assert call(k=192) == 2
+    assert call(m=-1) == 1
+    assert call(m=0) == 0
+    assert call(n=0) == 0
+    assert call(a_q=None) == 1
+    assert call(y=None) == 1
+    assert call(a_q=FAKE_ODD) == 3
+    assert call(bias=FAKE_ODD) == 3
+    assert call(s_w=ctypes.c_void_p(0x10002)) == 3

@@ -1,0 +1,126 @@
+"""GPU parity of the row-wise quantiser (bit-exact codes and scales)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import semi_structured_sparse_rowwise_b200 as S
+from semi_structured_sparse_rowwise_b200 import synthetic
+from gpu_pipeline import bf16_dev, ensure_library, requires_gpu, sample_indices
+
+pytestmark = [pytest.mark.gpu, requires_gpu]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_library()
+
+
+def _to_dev(x32, dtype):
+    t = torch.from_numpy(np.ascontiguousarray(x32))
+    return t.to(dtype).cuda()
+
+
+def _ref_from_dev(xd):
+    """Exact float32 widening of the device tensor's values, on the CPU."""
+    return xd.float().cpu().numpy()
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_exhaustive_bf16_sweep(fmt):
+    mx = np.float32(oracle.fp8_max(fmt))
+    v = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32)
+    v = v[np.isfinite(v) & (np.abs(v) <= mx)]
+    width = 256
+    v = np.concatenate([v, np.zeros((-v.size) % (width - 1), np.float32)])
+    body = v.reshape(-1, width - 1)
+    x = np.concatenate([np.full((body.shape[0], 1), mx, np.float32), body], axis=1)
+    xd = _to_dev(x, torch.bfloat16)
+    q, s = S.sfp8_quantize_rowwise(xd, fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+CASES = [
+    # rows, cols, torch dtype, distribution
+    (16, 128, torch.bfloat16, "normal"),
+    (1, 4096, torch.bfloat16, "normal"),
+    (4, 4096, torch.bfloat16, "normal"),
+    (16, 4096, torch.bfloat16, "normal"),
+    (37, 208, torch.bfloat16, "student_t3"),
+    (5, 16, torch.bfloat16, "normal"),
+    (1000, 4096, torch.bfloat16, "student_t3"),
+    (7, 16384, torch.bfloat16, "normal"),
+    (3, 65536, torch.bfloat16, "student_t3"),
+    (64, 4096, torch.float16, "normal"),
+    (33, 1024, torch.float32, "student_t3"),
+    (9, 16384, torch.float32, "normal"),
+    (3, 32768, torch.float32, "normal"),
+]
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("rows,cols,dtype,dist", CASES)
+def test_quantize_parity(rows, cols, dtype, dist, fmt):
+    bits = synthetic.activation(4242 + rows + cols, rows, cols, dist=dist, zero_row_frac=0.1)
+    x32 = oracle.bf16_bits_to_f32(bits) * np.float32(3.0)
+    xd = _to_dev(x32, dtype)
+    xr = _ref_from_dev(xd)
+    q, s = S.sfp8_quantize_rowwise(xd, fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(xr, fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_strided_input(fmt):
+    bits = synthetic.activation(99, 24, 512, dist="student_t3")
+    wide = bf16_dev(bits)
+    xd = wide[:, 128:384]                  # ld = 512, cols = 256
+    q, s = S.sfp8_quantize_rowwise(xd, fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(oracle.bf16_bits_to_f32(bits)[:, 128:384], fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_zero_and_negative_zero_rows():
+    x = np.zeros((4, 64), np.float32)
+    x[1, :] = -0.0
+    x[2, 7] = -0.0
+    x[3, 9] = 1e-30
+    for fmt in ("e4m3", "e5m2"):
+        q, s = S.sfp8_quantize_rowwise(_to_dev(x, torch.float32), fmt)
+        q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+        assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_empty_cols_and_rows():
+    xd = torch.empty((5, 0), dtype=torch.bfloat16, device="cuda")
+    q, s = S.sfp8_quantize_rowwise(xd, "e4m3")
+    _, s_ref = oracle.quantize_rowwise(np.zeros((5, 0), np.float32), "e4m3")
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    q, s = S.sfp8_quantize_rowwise(torch.empty((0, 64), dtype=torch.bfloat16, device="cuda"))
+    assert q.shape == (0, 64) and s.shape == (0,)
+
+
+@pytest.mark.parametrize("shape,dtype", [((65536, 4096), torch.bfloat16),
+                                         ((16384, 16384), torch.bfloat16),
+                                         ((65536, 4096), torch.float32)])
+def test_standalone_2p28_sampled(shape, dtype):
+    rows, cols = shape
+    g = torch.Generator(device="cpu").manual_seed(1004)
+    # the full tensor is generated on the CPU with numpy, like every input
+    bits = synthetic.activation(1004 * 100 + rows % 97, rows, cols, dist="normal")
+    xd = bf16_dev(bits).to(dtype)
+    q, s = S.sfp8_quantize_rowwise(xd, "e4m3")
+    sel = sample_indices(rows, 96, 5, must=(0, rows - 1))
+    q_ref, s_ref = oracle.quantize_rowwise(oracle.bf16_bits_to_f32(bits[sel]), "e4m3")
+    st = torch.from_numpy(sel).cuda()
+    assert np.array_equal(s.index_select(0, st).cpu().numpy().view(np.uint32),
+                          s_ref.view(np.uint32))
+    assert np.array_equal(q.index_select(0, st).cpu().numpy(), q_ref)
+    # every row: max |code| is reached (the amax element maps to +-FP8_MAX)
+    mags = (q & 0x7F).max(dim=1).values
+    assert bool((mags == 0x7E).all())
