@@ -186,6 +186,47 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Size of the scratch buffer built into the library for
+ * sfp8_sparse_linear_noalloc (per device that loads the library).
+ */
+#define SFP8_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * sfp8_sparse_linear for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that may not allocate at call time -- code replayed from a pre-built CUDA
+ * graph, runtimes whose allocator forbids cudaMalloc after start-up, or hosts
+ * that give the library nothing but its inputs and outputs.  It computes the
+ * same result as sfp8_sparse_linear (same kernel, same work split, so the
+ * same bits) but takes no workspace: the split-K scratch is a fixed
+ * SFP8_NOALLOC_SCRATCH_BYTES buffer compiled into the library, one per
+ * device, held until the process exits.  It calls no cudaMalloc/cudaFree or
+ * other allocating routine.
+ *
+ *  - Arguments, layouts and alignment as for sfp8_sparse_linear, minus the
+ *    workspace.
+ *  - Size limit: problems whose sfp8_sparse_linear_workspace_bytes(m, n, k)
+ *    exceeds SFP8_NOALLOC_SCRATCH_BYTES are rejected with SFP8_ERR_WORKSPACE
+ *    before anything is launched (on a 148-SM B200 this admits m <= 32 for
+ *    any n and k).
+ *  - The first call on a device looks up the buffer's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    outside any stream capture.
+ *  - All calls on a device share the one buffer, which keeps the previous
+ *    call's contents; each call clears the counters it needs (an async
+ *    memset on `stream`).  Calls that overlap on the GPU -- on different
+ *    streams, or on one stream inside concurrently replayed graphs -- race
+ *    on the buffer and give wrong results; serialise them.
+ */
+sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_dtype,
+                                       const float* s_a, int64_t m,
+                                       const void* values, const void* meta,
+                                       sfp8_dtype w_dtype, const float* s_w,
+                                       int64_t n, int64_t k, const void* bias,
+                                       void* y, void* stream);
+
+/*
  * Reads (and with clear != 0, resets) the current device's status word.
  * Synchronises the device first.  *flags receives SFP8_DEVICE_* bits.
  * Returns SFP8_ERR_TIMEOUT / SFP8_ERR_DEVICE_CHECK when such a bit is set,

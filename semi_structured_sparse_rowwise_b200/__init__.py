@@ -10,7 +10,8 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_compressed_values_bytes, sfp8_compressed_meta_bytes,
                       sfp8_compress_24, sfp8_decompress_24,
                       sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
-                      sfp8_sparse_linear, sfp8_read_device_status,
+                      sfp8_sparse_linear, sfp8_sparse_linear_noalloc,
+                      sfp8_read_device_status,
                       sfp8_status_string, sfp8_layout_version)
 from .layer import SparseFp8Linear
 
@@ -20,6 +21,6 @@ __all__ = [
     "sfp8_compressed_values_bytes", "sfp8_compressed_meta_bytes",
     "sfp8_compress_24", "sfp8_decompress_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
-    "sfp8_sparse_linear", "sfp8_read_device_status", "sfp8_status_string",
+    "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_read_device_status", "sfp8_status_string",
     "sfp8_layout_version", "SparseFp8Linear",
 ]

@@ -44,6 +44,9 @@ SIGNATURES = {
     "sfp8_sparse_linear": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _c_void_p, _i32,
                                   _c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _sz,
                                   _c_void_p]),
+    "sfp8_sparse_linear_noalloc": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p,
+                                          _c_void_p, _i32, _c_void_p, _i64, _i64, _c_void_p,
+                                          _c_void_p, _c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
     "sfp8_layout_version": (_i32, []),
@@ -232,6 +235,28 @@ def sfp8_sparse_linear(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k, bias
                                     _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
                                     workspace.numel(), _stream(a_q.device))
     _check(st, "sfp8_sparse_linear")
+    return out
+
+
+def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k,
+                               bias=None, out=None):
+    """sfp8_sparse_linear without a workspace, for callers that cannot
+    allocate device memory at call time (see include/sfp8.h): the library's
+    built-in scratch buffer is used instead.  `out` must be given by such a
+    caller; only when it is None does this wrapper allocate it with torch."""
+    lib = load_library()
+    _require_cuda(a_q, s_a, values, meta, s_w, bias)
+    if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
+        raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
+    m = a_q.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
+    with torch.cuda.device(a_q.device):
+        st = lib.sfp8_sparse_linear_noalloc(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
+                                            _ptr(values), _ptr(meta), DTYPE[_fp8_name(w_dtype)],
+                                            _ptr(s_w), n, k, _ptr(bias), _ptr(out),
+                                            _stream(a_q.device))
+    _check(st, "sfp8_sparse_linear_noalloc")
     return out
 
 

@@ -454,3 +454,115 @@ sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Sparse linear for callers that cannot allocate device memory.
+//
+// Some callers of this library run where no device allocation may happen at
+// call time: code that is replayed inside a pre-built CUDA graph, allocators
+// that forbid cudaMalloc after start-up, or hosts that hand the library only
+// its inputs and outputs.  For them the split-K scratch (partial sums and
+// per-tile counters) lives in a fixed buffer compiled into the library: one
+// copy per device that loads it, kept until the process exits.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = SFP8_NOALLOC_SCRATCH_BYTES;
+
+// In host code this name is only a stand-in; the device address is looked
+// up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[sfp8::kMaxDevices] = {};
+
+// Device address of the scratch buffer for the current device (set-up on
+// the first call per device).
+sfp8_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= sfp8::kMaxDevices)
+    return SFP8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return SFP8_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SFP8_OK;
+}
+
+}  // namespace
+
+extern "C" sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_dtype,
+                                                  const float* s_a, int64_t m,
+                                                  const void* values, const void* meta,
+                                                  sfp8_dtype w_dtype, const float* s_w,
+                                                  int64_t n, int64_t k, const void* bias,
+                                                  void* y, void* stream) {
+  if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
+  if (k == 0 || k % kStepK != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 31))
+    return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m == 0 || n == 0) return SFP8_OK;
+  if (a_q == nullptr || s_a == nullptr || values == nullptr || meta == nullptr ||
+      s_w == nullptr || y == nullptr)
+    return SFP8_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(values, 16) || !aligned(meta, 16) || !aligned(s_a, 4) ||
+      !aligned(s_w, 4) || !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
+    return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  const LinearPlan pl = make_plan(m, n, k, dev->num_sms);
+  if (pl.partial_bytes + pl.counter_bytes > kNoAllocScratchBytes) return SFP8_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != SFP8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* counters = static_cast<uint8_t*>(scratch) + pl.partial_bytes;
+  // The buffer keeps whatever the previous call left; the counters must
+  // start at zero (the partial sums are always written before being read).
+  if (cudaMemsetAsync(counters, 0, pl.counter_bytes, st) != cudaSuccess) return SFP8_ERR_CUDA;
+
+  CUtensorMap tw, ta;
+  const int64_t n_pad = sfp8_padded_rows(n);
+  s = encode_2d_u8(&tw, values, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n_pad),
+                   static_cast<uint64_t>(k / 2), kStepK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (s != SFP8_OK) return s;
+  s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
+                   static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SFP8_OK) return s;
+
+  LinearParams prm{};
+  prm.meta = static_cast<const uint8_t*>(meta);
+  prm.s_a = s_a;
+  prm.s_w = s_w;
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.y = static_cast<__nv_bfloat16*>(y);
+  prm.partials = static_cast<float*>(scratch);
+  prm.counters = reinterpret_cast<unsigned int*>(counters);
+  prm.m = static_cast<int>(m);
+  prm.n = static_cast<int>(n);
+  prm.k = static_cast<int>(k);
+  prm.m_tiles = pl.m_tiles;
+  prm.k_steps = pl.k_steps;
+  prm.tiles = pl.tiles;
+  prm.iters = pl.iters;
+  prm.grid = pl.grid;
+  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
+                                kTileN, static_cast<uint32_t>(pl.bn), true);
+  switch (pl.bn) {
+    case 16: return launch_linear_bn<16>(dev, 0, tw, ta, prm, st);
+    case 32: return launch_linear_bn<32>(dev, 1, tw, ta, prm, st);
+    case 64: return launch_linear_bn<64>(dev, 2, tw, ta, prm, st);
+    case 128: return launch_linear_bn<128>(dev, 3, tw, ta, prm, st);
+    default: return launch_linear_bn<256>(dev, 4, tw, ta, prm, st);
+  }
+}
