@@ -277,15 +277,15 @@ def run_ours(args):
     def prep():
         wp = S.sfp8_prune_24(w_dev)
         wq, sw = S.sfp8_quantize_rowwise(wp, "e4m3")
-        vals, meta = S.sfp8_compress_24(wq, "e4m3")
-        return wp, wq, sw, vals, meta
+        packed = S.sfp8_compress_24(wq, "e4m3")
+        return wp, wq, sw, packed
 
-    wp, wq, sw, vals, meta = prep()
+    wp, wq, sw, packed = prep()
     torch.cuda.synchronize(dev)
     off = {}
     for name, fn in (("prune_24", lambda: S.sfp8_prune_24(w_dev, out=wp)),
                      ("quantize_weight", lambda: S.sfp8_quantize_rowwise(wp, "e4m3", q=wq, scales=sw)),
-                     ("compress_24", lambda: S.sfp8_compress_24(wq, "e4m3", values=vals, meta=meta))):
+                     ("compress_24", lambda: S.sfp8_compress_24(wq, "e4m3", packed=packed))):
         for _ in range(3):
             fn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -306,8 +306,8 @@ def run_ours(args):
     }
 
     # ---- the step's buffers
-    copies = [(vals.clone(), meta.clone(), sw.clone()) for _ in range(WEIGHT_COPIES)]
-    del vals, meta
+    copies = [(packed.clone(), sw.clone()) for _ in range(WEIGHT_COPIES)]
+    del packed
     aq = torch.empty((m, k), dtype=torch.uint8, device=dev)
     sa = torch.empty((m,), dtype=torch.float32, device=dev)
     ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(WEIGHT_COPIES)]
@@ -317,8 +317,8 @@ def run_ours(args):
         S.sfp8_quantize_rowwise(x_dev, "e4m3", q=aq, scales=sa)
 
     def gemm(j):
-        v, mt, s = copies[j % WEIGHT_COPIES]
-        S.sfp8_sparse_linear(aq, "e4m3", sa, v, mt, "e4m3", s, n, k, out=ys[j % WEIGHT_COPIES],
+        pk, s = copies[j % WEIGHT_COPIES]
+        S.sfp8_sparse_linear(aq, "e4m3", sa, pk, "e4m3", s, n, k, out=ys[j % WEIGHT_COPIES],
                              workspace=ws)
 
     def step(j):
@@ -382,7 +382,7 @@ def run_ours(args):
         traffic = NCU_TRAFFIC["bytes_per_launch"]
 
     # ---- end to end through the layer, host buffers, eager calls
-    layer = S.SparseFp8Linear.from_compressed(copies[0][0], copies[0][1], copies[0][2], n, k)
+    layer = S.SparseFp8Linear.from_compressed(copies[0][0], copies[0][1], n, k)
     x_host = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(
         torch.bfloat16).pin_memory()
     y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
@@ -418,8 +418,8 @@ def run_ours(args):
 
             def step2(j, x2=x2, aq2=aq2, sa2=sa2, y2=y2, ws2=ws2, m2=m2):
                 S.sfp8_quantize_rowwise(x2, "e4m3", q=aq2, scales=sa2)
-                v, mt, s = copies[j % WEIGHT_COPIES]
-                S.sfp8_sparse_linear(aq2, "e4m3", sa2, v, mt, "e4m3", s, n, k, out=y2,
+                pk, s = copies[j % WEIGHT_COPIES]
+                S.sfp8_sparse_linear(aq2, "e4m3", sa2, pk, "e4m3", s, n, k, out=y2,
                                      workspace=ws2)
             for j in range(args.warmup):
                 step2(j)

@@ -67,7 +67,7 @@ typedef enum {
 #define SFP8_DEVICE_CHECK_FAIL  0x2u  /* a device-side check failed          */
 
 /* Version of the compressed-weight layout written by sfp8_compress_24. */
-#define SFP8_LAYOUT_VERSION 1
+#define SFP8_LAYOUT_VERSION 3
 
 /*
  * Dynamic row-wise FP8 quantisation (the activation path of item 4; also
@@ -110,49 +110,54 @@ sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows,
                           int64_t cols, int64_t ld, void* out, void* stream);
 
 /*
- * Compressed-weight sizes for an [n, k] FP8 weight (k % 128 == 0).
- * Rows are padded to n_pad = ceil(n / 128) * 128.
- *   values: n_pad * k / 2 bytes;  meta: n_pad * k / 8 bytes.
+ * Size of the compressed (packed) weight for an [n, k] FP8 weight
+ * (k % 128 == 0): n_pad * k * 5/8 bytes with n_pad = ceil(n / 128) * 128.
  */
 int64_t sfp8_padded_rows(int64_t n);
-size_t sfp8_compressed_values_bytes(int64_t n, int64_t k);
-size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k);
+size_t sfp8_compressed_bytes(int64_t n, int64_t k);
 
 /*
  * 2:4 compression of an FP8 weight (item 1's converter, with item 3's rule
  * that -0.0 is a zero).  Per group g of four codes along k: keep the two of
  * largest magnitude (ties to the lower index; -0.0 ranks as 0), emit the two
  * source codes unchanged, lower index first, and the index nibble
- * i0 | (i1 << 2).  Layout (version 1):
- *   values: [n_pad, k/2] bytes, row-major, the kept codes group by group.
- *   meta:   2048-byte tiles; tile (nt, kt) (nt < n_pad/128, kt < k/128) at
- *           byte (nt*(k/128) + kt)*2048; inside, weight row 128*nt + r at
- *           byte 16*r, byte b holding the nibble of group 32*kt + 2b in bits
- *           0..3 and of group 32*kt + 2b + 1 in bits 4..7.
+ * i0 | (i1 << 2).
+ *
+ * Layout (version 3): one buffer of 10240-byte tiles; tile t = nt*(k/128)+kt
+ * covers weight rows 128*nt .. 128*nt+127 and k columns 128*kt .. 128*kt+127
+ * and starts at byte 10240*t:
+ *   bytes 0 .. 8191: kept values.  Row r of the tile at byte 64*r holds the
+ *           row's 64 kept codes (two per group, lower index first) as four
+ *           16-byte chunks, chunk c at position c ^ ((r >> 1) & 3).
+ *   bytes 8192 .. 10239: index metadata.  Row r at byte 8192 + 16*r; byte b
+ *           holds the nibble of group 32*kt + 2b in bits 0..3 and of group
+ *           32*kt + 2b + 1 in bits 4..7.
  *   Rows n..n_pad-1: value 0x00 and nibble 0x4 everywhere.
+ * (One tile is exactly what one k step of the GEMM needs in shared memory,
+ * values already in the tensor core's 64-byte-swizzled form, so the GEMM
+ * streams the weight with one contiguous copy per pipeline stage.)
  *
  *  w_q     device, [n, k] FP8 codes (w_dtype E4M3 or E5M2), row stride k,
  *          16-byte aligned.  NaN codes are outside the contract.
- *  values, meta  device, sizes above, 16-byte aligned.
+ *  packed  device, sfp8_compressed_bytes(n, k) bytes, 16-byte aligned.
  */
 sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n,
-                             int64_t k, void* values, void* meta,
-                             void* stream);
+                             int64_t k, void* packed, void* stream);
 
 /*
  * Inverse of sfp8_compress_24 (a checking aid): writes the dense [n, k]
  * codes, 0x00 in dropped slots.  w_q 16-byte aligned, row stride k.
  * An invalid nibble sets SFP8_DEVICE_CHECK_FAIL in the device status word.
  */
-sfp8_status sfp8_decompress_24(const void* values, const void* meta,
-                               int64_t n, int64_t k, void* w_q, void* stream);
+sfp8_status sfp8_decompress_24(const void* packed, int64_t n, int64_t k,
+                               void* w_q, void* stream);
 
 /*
  * Workspace for sfp8_sparse_linear on the current device (split-K partial
- * sums and per-tile counters).  The counters part must be zero before the
- * first call that uses a workspace; every call leaves it zero again (clear it
- * again after a call that reported a device error).  sfp8_workspace_clear
- * zeroes a workspace on a stream.
+ * sums and per-tile counters); 0 when the chosen work split needs none.  The
+ * counters part must be zero before the first call that uses a workspace;
+ * every call leaves it zero again (clear it again after a call that reported
+ * a device error).  sfp8_workspace_clear zeroes a workspace on a stream.
  */
 size_t sfp8_sparse_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 sfp8_status sfp8_workspace_clear(void* workspace, size_t workspace_bytes,
@@ -168,21 +173,26 @@ sfp8_status sfp8_workspace_clear(void* workspace, size_t workspace_bytes,
  *  a_q     device, [m, k] FP8 codes (a_dtype E4M3 or E5M2), row stride k,
  *          16-byte aligned.
  *  s_a     device, [m] float32.
- *  values, meta  device, from sfp8_compress_24 for an [n, k] weight of
- *          w_dtype (E4M3 or E5M2).
+ *  packed  device, from sfp8_compress_24 for an [n, k] weight of w_dtype
+ *          (E4M3 or E5M2).
  *  s_w     device, [n] float32.
  *  bias    device, [n] bf16, or NULL for none.
  *  y       device, [m, n] bf16, row stride n.
- *  workspace  device, >= sfp8_sparse_linear_workspace_bytes(m, n, k) bytes,
- *          16-byte aligned, counters zero (see above).
+ *  workspace  device, >= sfp8_sparse_linear_workspace_bytes(m, n, k) bytes
+ *          (may be NULL when that is 0), 16-byte aligned, counters zero.
  *  k % 128 == 0, k > 0; m, n >= 0.
+ *
+ * The call is launched as a programmatic dependent of the preceding kernel on
+ * the stream: it streams the first weight tiles before waiting for that
+ * kernel to finish, and reads a_q, s_a, bias only after.  So `packed` and
+ * `s_w` must not be written by a kernel that lets its dependents launch
+ * early (none of this library's kernels writes them that way).
  */
 sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
                                const float* s_a, int64_t m,
-                               const void* values, const void* meta,
-                               sfp8_dtype w_dtype, const float* s_w,
-                               int64_t n, int64_t k, const void* bias,
-                               void* y, void* workspace,
+                               const void* packed, sfp8_dtype w_dtype,
+                               const float* s_w, int64_t n, int64_t k,
+                               const void* bias, void* y, void* workspace,
                                size_t workspace_bytes, void* stream);
 
 /*
@@ -221,8 +231,8 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
  */
 sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_dtype,
                                        const float* s_a, int64_t m,
-                                       const void* values, const void* meta,
-                                       sfp8_dtype w_dtype, const float* s_w,
+                                       const void* packed, sfp8_dtype w_dtype,
+                                       const float* s_w,
                                        int64_t n, int64_t k, const void* bias,
                                        void* y, void* stream);
 

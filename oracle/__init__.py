@@ -39,7 +39,7 @@ from .fp8 import (E4M3, E5M2, FORMATS, decode_table, decode, fp8_max,
 from .quantize import quantize_rowwise, GUARD_AMAX
 from .prune import prune_24
 from .compress import compress_24, decompress_24, NIBBLES_VALID
-from .layout import unpack_physical, padded_rows, values_bytes, meta_bytes
+from .layout import unpack_physical, padded_rows, packed_bytes
 from .linear import sparse_linear_ref, acceptance_bound, check_linear
 
 __all__ = [
@@ -47,6 +47,6 @@ __all__ = [
     "encode_rne_sat", "bf16_bits_to_f32", "f16_bits_to_f32", "round_to_bf16",
     "quantize_rowwise", "GUARD_AMAX", "prune_24", "compress_24",
     "decompress_24", "NIBBLES_VALID", "unpack_physical", "padded_rows",
-    "values_bytes", "meta_bytes", "sparse_linear_ref", "acceptance_bound",
+    "packed_bytes", "sparse_linear_ref", "acceptance_bound",
     "check_linear",
 ]

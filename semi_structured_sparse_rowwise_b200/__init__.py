@@ -7,7 +7,7 @@ class on top of it, and the seeded synthetic-input generators.
 
 from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_quantize_rowwise, sfp8_prune_24, sfp8_padded_rows,
-                      sfp8_compressed_values_bytes, sfp8_compressed_meta_bytes,
+                      sfp8_compressed_bytes,
                       sfp8_compress_24, sfp8_decompress_24,
                       sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
                       sfp8_sparse_linear, sfp8_sparse_linear_noalloc,
@@ -18,7 +18,7 @@ from .layer import SparseFp8Linear
 __all__ = [
     "Sfp8Error", "load_library", "library_path", "new_workspace",
     "sfp8_quantize_rowwise", "sfp8_prune_24", "sfp8_padded_rows",
-    "sfp8_compressed_values_bytes", "sfp8_compressed_meta_bytes",
+    "sfp8_compressed_bytes",
     "sfp8_compress_24", "sfp8_decompress_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
     "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_read_device_status", "sfp8_status_string",

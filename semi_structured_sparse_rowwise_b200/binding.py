@@ -35,17 +35,16 @@ SIGNATURES = {
                                      _c_void_p, _c_void_p]),
     "sfp8_prune_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_padded_rows": (_i64, [_i64]),
-    "sfp8_compressed_values_bytes": (_sz, [_i64, _i64]),
-    "sfp8_compressed_meta_bytes": (_sz, [_i64, _i64]),
-    "sfp8_compress_24": (_i32, [_c_void_p, _i32, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
-    "sfp8_decompress_24": (_i32, [_c_void_p, _c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "sfp8_compressed_bytes": (_sz, [_i64, _i64]),
+    "sfp8_compress_24": (_i32, [_c_void_p, _i32, _i64, _i64, _c_void_p, _c_void_p]),
+    "sfp8_decompress_24": (_i32, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_sparse_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "sfp8_workspace_clear": (_i32, [_c_void_p, _sz, _c_void_p]),
-    "sfp8_sparse_linear": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _c_void_p, _i32,
+    "sfp8_sparse_linear": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _i32,
                                   _c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p, _sz,
                                   _c_void_p]),
     "sfp8_sparse_linear_noalloc": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p,
-                                          _c_void_p, _i32, _c_void_p, _i64, _i64, _c_void_p,
+                                          _i32, _c_void_p, _i64, _i64, _c_void_p,
                                           _c_void_p, _c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
@@ -153,42 +152,34 @@ def sfp8_padded_rows(n):
     return int(load_library().sfp8_padded_rows(n))
 
 
-def sfp8_compressed_values_bytes(n, k):
-    return int(load_library().sfp8_compressed_values_bytes(n, k))
+def sfp8_compressed_bytes(n, k):
+    return int(load_library().sfp8_compressed_bytes(n, k))
 
 
-def sfp8_compressed_meta_bytes(n, k):
-    return int(load_library().sfp8_compressed_meta_bytes(n, k))
-
-
-def sfp8_compress_24(w_q, w_dtype="e4m3", values=None, meta=None):
-    """w_q [n, k] uint8 FP8 codes -> (values, meta) in the library's layout."""
+def sfp8_compress_24(w_q, w_dtype="e4m3", packed=None):
+    """w_q [n, k] uint8 FP8 codes -> packed compressed weight (layout v3)."""
     lib = load_library()
     _require_cuda(w_q)
     if w_q.dim() != 2 or not w_q.is_contiguous() or w_q.dtype != torch.uint8:
         raise ValueError("w_q must be a contiguous 2-D uint8 tensor")
     n, k = w_q.shape
-    if values is None:
-        values = torch.empty((lib.sfp8_compressed_values_bytes(n, k),), dtype=torch.uint8,
+    if packed is None:
+        packed = torch.empty((lib.sfp8_compressed_bytes(n, k),), dtype=torch.uint8,
                              device=w_q.device)
-    if meta is None:
-        meta = torch.empty((lib.sfp8_compressed_meta_bytes(n, k),), dtype=torch.uint8,
-                           device=w_q.device)
     with torch.cuda.device(w_q.device):
-        st = lib.sfp8_compress_24(_ptr(w_q), DTYPE[_fp8_name(w_dtype)], n, k, _ptr(values),
-                                  _ptr(meta), _stream(w_q.device))
+        st = lib.sfp8_compress_24(_ptr(w_q), DTYPE[_fp8_name(w_dtype)], n, k, _ptr(packed),
+                                  _stream(w_q.device))
     _check(st, "sfp8_compress_24")
-    return values, meta
+    return packed
 
 
-def sfp8_decompress_24(values, meta, n, k, out=None):
+def sfp8_decompress_24(packed, n, k, out=None):
     lib = load_library()
-    _require_cuda(values, meta)
+    _require_cuda(packed)
     if out is None:
-        out = torch.empty((n, k), dtype=torch.uint8, device=values.device)
-    with torch.cuda.device(values.device):
-        st = lib.sfp8_decompress_24(_ptr(values), _ptr(meta), n, k, _ptr(out),
-                                    _stream(values.device))
+        out = torch.empty((n, k), dtype=torch.uint8, device=packed.device)
+    with torch.cuda.device(packed.device):
+        st = lib.sfp8_decompress_24(_ptr(packed), n, k, _ptr(out), _stream(packed.device))
     _check(st, "sfp8_decompress_24")
     return out
 
@@ -213,11 +204,11 @@ def sfp8_workspace_clear(workspace):
     _check(st, "sfp8_workspace_clear")
 
 
-def sfp8_sparse_linear(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k, bias=None,
+def sfp8_sparse_linear(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bias=None,
                        out=None, workspace=None):
     """y [m, n] bf16 = (s_a s_w^T) * (A_q . W_q^T) + bias."""
     lib = load_library()
-    _require_cuda(a_q, s_a, values, meta, s_w, bias)
+    _require_cuda(a_q, s_a, packed, s_w, bias)
     if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
         raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
     m = a_q.shape[0]
@@ -231,21 +222,21 @@ def sfp8_sparse_linear(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k, bias
         raise ValueError("bias must be bfloat16")
     with torch.cuda.device(a_q.device):
         st = lib.sfp8_sparse_linear(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
-                                    _ptr(values), _ptr(meta), DTYPE[_fp8_name(w_dtype)],
+                                    _ptr(packed), DTYPE[_fp8_name(w_dtype)],
                                     _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
                                     workspace.numel(), _stream(a_q.device))
     _check(st, "sfp8_sparse_linear")
     return out
 
 
-def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n, k,
+def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k,
                                bias=None, out=None):
     """sfp8_sparse_linear without a workspace, for callers that cannot
     allocate device memory at call time (see include/sfp8.h): the library's
     built-in scratch buffer is used instead.  `out` must be given by such a
     caller; only when it is None does this wrapper allocate it with torch."""
     lib = load_library()
-    _require_cuda(a_q, s_a, values, meta, s_w, bias)
+    _require_cuda(a_q, s_a, packed, s_w, bias)
     if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
         raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
     m = a_q.shape[0]
@@ -253,7 +244,7 @@ def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, values, meta, w_dtype, s_w, n,
         out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
     with torch.cuda.device(a_q.device):
         st = lib.sfp8_sparse_linear_noalloc(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
-                                            _ptr(values), _ptr(meta), DTYPE[_fp8_name(w_dtype)],
+                                            _ptr(packed), DTYPE[_fp8_name(w_dtype)],
                                             _ptr(s_w), n, k, _ptr(bias), _ptr(out),
                                             _stream(a_q.device))
     _check(st, "sfp8_sparse_linear_noalloc")

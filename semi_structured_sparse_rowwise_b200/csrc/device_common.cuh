@@ -86,6 +86,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+// Atomic add with release and acquire semantics at GPU scope; returns the
+// previous value.
+__device__ __forceinline__ unsigned int atomic_add_acq_rel_gpu(unsigned int* addr,
+                                                               unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(addr), "r"(v)
+               : "memory");
+  return old;
+}
+
+__device__ __forceinline__ unsigned int load_acquire_gpu(const unsigned int* addr) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------- TMA / bulk
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* desc) {

@@ -9,6 +9,11 @@
 // with warp shuffles (and shared memory across warps when TPR > 32), then
 // converts from the registers.  Rows too long for the register tile use a
 // two-sweep variant that re-reads the row (from L2).
+//
+// The kernels are launched as programmatic dependents: they let their own
+// dependents (the GEMM) launch at once, then wait for the preceding grid to
+// complete before reading x or writing q and the scales -- the preceding
+// grid may be the GEMM of the previous call that still reads them.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -135,6 +140,7 @@ __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
     quantize_rowwise_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* __restrict__ q, float* __restrict__ scales) {
   grid_dependents_launch();
+  grid_dependency_wait();
   using Tr = InputTraits<T>;
   constexpr int P = Tr::kPerVec;
   __shared__ float red[32];
@@ -183,6 +189,7 @@ __global__ void __launch_bounds__(1024)
                                  int64_t ld, uint8_t* __restrict__ q,
                                  float* __restrict__ scales) {
   grid_dependents_launch();
+  grid_dependency_wait();
   using Tr = InputTraits<T>;
   constexpr int P = Tr::kPerVec;
   __shared__ float red[32];
@@ -215,6 +222,7 @@ __global__ void __launch_bounds__(1024)
 template <int kFmt>
 __global__ void quantize_empty_rows_kernel(int64_t rows, float* __restrict__ scales) {
   grid_dependents_launch();
+  grid_dependency_wait();
   const int64_t r = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (r < rows) scales[r] = __fdiv_rn(kGuardAmax, Fp8Out<kFmt>::kMax);
 }

@@ -24,7 +24,7 @@ struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
   int num_sms = 0;
-  bool smem_attr_set[8] = {};
+  bool smem_attr_set[16] = {};
 };
 
 std::mutex g_mutex;
@@ -97,6 +97,29 @@ inline int elem_size(sfp8_dtype t) {
 inline bool is_fp8(sfp8_dtype t) { return t == SFP8_E4M3 || t == SFP8_E5M2; }
 inline bool is_wide(sfp8_dtype t) { return t == SFP8_BF16 || t == SFP8_F16 || t == SFP8_F32; }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous grid on the stream finishes; it waits for it (griddepcontrol)
+// before touching memory.
+template <typename Kernel, typename... Args>
+sfp8_status launch_dependent(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return SFP8_ERR_CUDA;
+  }
+  return SFP8_OK;
+}
+
 // ------------------------------------------------------------------ quantise
 
 template <typename T, int kFmt>
@@ -106,28 +129,30 @@ sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   uint8_t* qp = static_cast<uint8_t*>(q);
   if (cols == 0) {
     const int64_t blocks = (rows + 255) / 256;
-    quantize_empty_rows_kernel<kFmt><<<static_cast<unsigned>(blocks), 256, 0, st>>>(rows, scales);
-    return launch_status();
+    return launch_dependent(quantize_empty_rows_kernel<kFmt>, dim3(static_cast<unsigned>(blocks)),
+                            dim3(256), 0, st, rows, scales);
   }
   constexpr int P = InputTraits<T>::kPerVec;
   const int64_t nvec = cols / P;
   constexpr int kChunks = 8;
   if (nvec <= 32 * kChunks) {
     const int64_t blocks = (rows + 7) / 8;
-    quantize_rowwise_kernel<T, kFmt, 32, kChunks>
-        <<<static_cast<unsigned>(blocks), 256, 0, st>>>(xp, rows, cols, ld, qp, scales);
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, kChunks>,
+                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
+                            ld, qp, scales);
   } else if (nvec <= 128 * kChunks) {
     const int64_t blocks = (rows + 1) / 2;
-    quantize_rowwise_kernel<T, kFmt, 128, kChunks>
-        <<<static_cast<unsigned>(blocks), 256, 0, st>>>(xp, rows, cols, ld, qp, scales);
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 128, kChunks>,
+                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
+                            ld, qp, scales);
   } else if (nvec <= 512 * kChunks) {
-    quantize_rowwise_kernel<T, kFmt, 512, kChunks>
-        <<<static_cast<unsigned>(rows), 512, 0, st>>>(xp, rows, cols, ld, qp, scales);
-  } else {
-    quantize_rowwise_long_kernel<T, kFmt>
-        <<<static_cast<unsigned>(rows), 1024, 0, st>>>(xp, rows, cols, ld, qp, scales);
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 512, kChunks>,
+                            dim3(static_cast<unsigned>(rows)), dim3(512), 0, st, xp, rows, cols,
+                            ld, qp, scales);
   }
-  return launch_status();
+  return launch_dependent(quantize_rowwise_long_kernel<T, kFmt>,
+                          dim3(static_cast<unsigned>(rows)), dim3(1024), 0, st, xp, rows, cols,
+                          ld, qp, scales);
 }
 
 template <typename T>
@@ -141,9 +166,12 @@ sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64
 
 struct LinearPlan {
   int bn;
+  int ks;               // k steps per pipeline stage
+  int whole_tiles;      // 1: each CTA takes whole tiles; 0: stream-K
   int grid;
   int m_tiles;
   int k_steps;
+  int units;            // stages per tile
   long long n_tiles;
   long long tiles;
   long long iters;
@@ -164,22 +192,41 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   pl.bn = choose_bn(m);
   pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
   pl.k_steps = static_cast<int>(k / kStepK);
+  // Two k steps per stage (one 20 KB weight copy) when the stage stays small.
+  pl.ks = (pl.bn <= 64 && pl.k_steps % 2 == 0) ? 2 : 1;
+  pl.units = pl.k_steps / pl.ks;
   pl.n_tiles = (n + kTileN - 1) / kTileN;
   pl.tiles = pl.n_tiles * pl.m_tiles;
-  pl.iters = pl.tiles * pl.k_steps;
-  pl.grid = static_cast<int>(pl.iters < num_sms ? pl.iters : num_sms);
-  if (pl.grid < 1) pl.grid = 1;
-  pl.partial_bytes = static_cast<size_t>(pl.grid) * 2 * pl.bn * kTileN * sizeof(float);
-  pl.partial_bytes = (pl.partial_bytes + 255) & ~static_cast<size_t>(255);
-  pl.counter_bytes = static_cast<size_t>(pl.tiles) * 4 * sizeof(unsigned int);
+  pl.iters = pl.tiles * pl.units;
+  if (pl.bn <= 32) {
+    // Bandwidth-bound: whole tiles (no split-K fix-up) once there are enough
+    // of them to keep three quarters of the SMs streaming.
+    pl.whole_tiles = pl.tiles * 4 >= 3LL * num_sms ? 1 : 0;
+  } else {
+    // Compute-bound: whole tiles when the last wave is nearly full.
+    const long long waves = (pl.tiles + num_sms - 1) / num_sms;
+    pl.whole_tiles = (pl.tiles >= num_sms && pl.tiles * 10 >= 9 * waves * num_sms) ? 1 : 0;
+  }
+  if (pl.whole_tiles) {
+    pl.grid = static_cast<int>(pl.tiles < num_sms ? pl.tiles : num_sms);
+    pl.partial_bytes = 0;
+    pl.counter_bytes = 0;
+  } else {
+    pl.grid = static_cast<int>(pl.iters < num_sms ? pl.iters : num_sms);
+    if (pl.grid < 1) pl.grid = 1;
+    pl.partial_bytes = static_cast<size_t>(pl.grid) * 2 * pl.bn * kTileN * sizeof(float);
+    pl.partial_bytes = (pl.partial_bytes + 255) & ~static_cast<size_t>(255);
+    pl.counter_bytes = static_cast<size_t>(pl.tiles) * 4 * sizeof(unsigned int);
+  }
   return pl;
 }
 
-template <int BN>
-sfp8_status launch_linear_bn(DeviceInfo* dev, int slot, const CUtensorMap& tw,
-                             const CUtensorMap& ta, const LinearParams& prm, cudaStream_t st) {
-  using Cfg = LinearCfg<BN>;
-  auto kern = sparse_linear_kernel<BN>;
+template <int BN, int KS>
+sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const LinearParams& prm,
+                              cudaStream_t st) {
+  using Cfg = LinearCfg<BN, KS>;
+  auto kern = sparse_linear_kernel<BN, KS>;
+  const int slot = (BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 2 + (KS - 1);
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev->smem_attr_set[slot]) {
@@ -189,21 +236,7 @@ sfp8_status launch_linear_bn(DeviceInfo* dev, int slot, const CUtensorMap& tw,
       dev->smem_attr_set[slot] = true;
     }
   }
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(prm.grid);
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tw, ta, prm) != cudaSuccess) {
-    cudaGetLastError();
-    return SFP8_ERR_CUDA;
-  }
-  return SFP8_OK;
+  return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, ta, prm);
 }
 
 sfp8_status encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
@@ -220,6 +253,81 @@ sfp8_status encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uin
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
+}
+
+// Validation shared by the sparse-linear entry points (everything except the
+// workspace); on success fills *plan for the current device.
+sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_a, int64_t m,
+                            const void* packed, sfp8_dtype w_dtype, const float* s_w, int64_t n,
+                            int64_t k, const void* bias, const void* y, DeviceInfo** dev,
+                            LinearPlan* plan, bool* empty) {
+  *empty = false;
+  if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
+  if (k == 0 || k % kStepK != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 31))
+    return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (m == 0 || n == 0) {
+    *empty = true;
+    return SFP8_OK;
+  }
+  if (a_q == nullptr || s_a == nullptr || packed == nullptr || s_w == nullptr || y == nullptr)
+    return SFP8_ERR_INVALID_ARG;
+  if (!aligned(a_q, 16) || !aligned(packed, 16) || !aligned(s_a, 4) || !aligned(s_w, 4) ||
+      !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
+    return SFP8_ERR_MISALIGNED;
+  sfp8_status s = current_device(dev);
+  if (s != SFP8_OK) return s;
+  *plan = make_plan(m, n, k, (*dev)->num_sms);
+  return SFP8_OK;
+}
+
+// Encodes the activation map and launches the GEMM for a validated plan.
+sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
+                          sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
+                          sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
+                          const void* bias, void* y, float* partials, unsigned int* counters,
+                          cudaStream_t st) {
+  CUtensorMap ta;
+  sfp8_status s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
+                               static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SFP8_OK) return s;
+  LinearParams prm{};
+  prm.packed = static_cast<const uint8_t*>(packed);
+  prm.s_a = s_a;
+  prm.s_w = s_w;
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.y = static_cast<__nv_bfloat16*>(y);
+  prm.partials = partials;
+  prm.counters = counters;
+  prm.m = static_cast<int>(m);
+  prm.n = static_cast<int>(n);
+  prm.k = static_cast<int>(k);
+  prm.m_tiles = pl.m_tiles;
+  prm.k_steps = pl.k_steps;
+  prm.units = pl.units;
+  prm.tiles = pl.tiles;
+  prm.iters = pl.iters;
+  prm.grid = pl.grid;
+  prm.whole_tiles = pl.whole_tiles;
+  // MMA A operand = weight, B operand = activation.
+  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
+                                kTileN, static_cast<uint32_t>(pl.bn), true);
+  if (pl.ks == 2) {
+    switch (pl.bn) {
+      case 16: return launch_linear_cfg<16, 2>(dev, ta, prm, st);
+      case 32: return launch_linear_cfg<32, 2>(dev, ta, prm, st);
+      default: return launch_linear_cfg<64, 2>(dev, ta, prm, st);
+    }
+  }
+  switch (pl.bn) {
+    case 16: return launch_linear_cfg<16, 1>(dev, ta, prm, st);
+    case 32: return launch_linear_cfg<32, 1>(dev, ta, prm, st);
+    case 64: return launch_linear_cfg<64, 1>(dev, ta, prm, st);
+    case 128: return launch_linear_cfg<128, 1>(dev, ta, prm, st);
+    default: return launch_linear_cfg<256, 1>(dev, ta, prm, st);
+  }
 }
 
 }  // namespace
@@ -252,14 +360,9 @@ int64_t sfp8_padded_rows(int64_t n) {
   return ((n + kTileN - 1) / kTileN) * kTileN;
 }
 
-size_t sfp8_compressed_values_bytes(int64_t n, int64_t k) {
+size_t sfp8_compressed_bytes(int64_t n, int64_t k) {
   if (n < 0 || k < 0) return 0;
-  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k / 2);
-}
-
-size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k) {
-  if (n < 0 || k < 0) return 0;
-  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k / 8);
+  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k) * 5 / 8;
 }
 
 sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype, int64_t rows, int64_t cols,
@@ -319,39 +422,37 @@ sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows, int64_t
 }
 
 sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n, int64_t k,
-                             void* values, void* meta, void* stream) {
+                             void* packed, void* stream) {
   if (!is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
   if (n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
   if (k % kStepK != 0 || k == 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
   if (n == 0) return SFP8_OK;
   if (k / kStepK > 65535 || sfp8_padded_rows(n) / kTileN > 65535) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (w_q == nullptr || values == nullptr || meta == nullptr) return SFP8_ERR_INVALID_ARG;
-  if (!aligned(w_q, 16) || !aligned(values, 16) || !aligned(meta, 16)) return SFP8_ERR_MISALIGNED;
+  if (w_q == nullptr || packed == nullptr) return SFP8_ERR_INVALID_ARG;
+  if (!aligned(w_q, 16) || !aligned(packed, 16)) return SFP8_ERR_MISALIGNED;
   DeviceInfo* dev = nullptr;
   sfp8_status s = current_device(&dev);
   if (s != SFP8_OK) return s;
   dim3 grid(static_cast<unsigned>(k / kStepK), static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
   compress24_kernel<<<grid, 512, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint8_t*>(w_q), n, k, static_cast<uint8_t*>(values),
-      static_cast<uint8_t*>(meta));
+      static_cast<const uint8_t*>(w_q), n, k, static_cast<uint8_t*>(packed));
   return launch_status();
 }
 
-sfp8_status sfp8_decompress_24(const void* values, const void* meta, int64_t n, int64_t k,
-                               void* w_q, void* stream) {
+sfp8_status sfp8_decompress_24(const void* packed, int64_t n, int64_t k, void* w_q,
+                               void* stream) {
   if (n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
   if (k % kStepK != 0 || k == 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
   if (n == 0) return SFP8_OK;
   if (k / kStepK > 65535 || sfp8_padded_rows(n) / kTileN > 65535) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (w_q == nullptr || values == nullptr || meta == nullptr) return SFP8_ERR_INVALID_ARG;
-  if (!aligned(w_q, 16) || !aligned(values, 16) || !aligned(meta, 16)) return SFP8_ERR_MISALIGNED;
+  if (w_q == nullptr || packed == nullptr) return SFP8_ERR_INVALID_ARG;
+  if (!aligned(w_q, 16) || !aligned(packed, 16)) return SFP8_ERR_MISALIGNED;
   DeviceInfo* dev = nullptr;
   sfp8_status s = current_device(&dev);
   if (s != SFP8_OK) return s;
   dim3 grid(static_cast<unsigned>(k / kStepK), static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
   decompress24_kernel<<<grid, 512, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint8_t*>(values), static_cast<const uint8_t*>(meta), n, k,
-      static_cast<uint8_t*>(w_q));
+      static_cast<const uint8_t*>(packed), n, k, static_cast<uint8_t*>(w_q));
   return launch_status();
 }
 
@@ -375,66 +476,24 @@ sfp8_status sfp8_workspace_clear(void* workspace, size_t workspace_bytes, void* 
 }
 
 sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_a, int64_t m,
-                               const void* values, const void* meta, sfp8_dtype w_dtype,
-                               const float* s_w, int64_t n, int64_t k, const void* bias, void* y,
-                               void* workspace, size_t workspace_bytes, void* stream) {
-  if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
-  if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
-  if (k == 0 || k % kStepK != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 31))
-    return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (m == 0 || n == 0) return SFP8_OK;
-  if (a_q == nullptr || s_a == nullptr || values == nullptr || meta == nullptr ||
-      s_w == nullptr || y == nullptr)
-    return SFP8_ERR_INVALID_ARG;
-  if (!aligned(a_q, 16) || !aligned(values, 16) || !aligned(meta, 16) || !aligned(s_a, 4) ||
-      !aligned(s_w, 4) || !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
-    return SFP8_ERR_MISALIGNED;
+                               const void* packed, sfp8_dtype w_dtype, const float* s_w,
+                               int64_t n, int64_t k, const void* bias, void* y, void* workspace,
+                               size_t workspace_bytes, void* stream) {
   DeviceInfo* dev = nullptr;
-  sfp8_status s = current_device(&dev);
-  if (s != SFP8_OK) return s;
-  const LinearPlan pl = make_plan(m, n, k, dev->num_sms);
-  if (workspace == nullptr || workspace_bytes < pl.partial_bytes + pl.counter_bytes)
-    return SFP8_ERR_WORKSPACE;
-  if (!aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
-
-  CUtensorMap tw, ta;
-  const int64_t n_pad = sfp8_padded_rows(n);
-  s = encode_2d_u8(&tw, values, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n_pad),
-                   static_cast<uint64_t>(k / 2), kStepK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (s != SFP8_OK) return s;
-  s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
-                   static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
-                   CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != SFP8_OK) return s;
-
-  LinearParams prm{};
-  prm.meta = static_cast<const uint8_t*>(meta);
-  prm.s_a = s_a;
-  prm.s_w = s_w;
-  prm.bias = static_cast<const __nv_bfloat16*>(bias);
-  prm.y = static_cast<__nv_bfloat16*>(y);
-  prm.partials = static_cast<float*>(workspace);
-  prm.counters = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(workspace) + pl.partial_bytes);
-  prm.m = static_cast<int>(m);
-  prm.n = static_cast<int>(n);
-  prm.k = static_cast<int>(k);
-  prm.m_tiles = pl.m_tiles;
-  prm.k_steps = pl.k_steps;
-  prm.tiles = pl.tiles;
-  prm.iters = pl.iters;
-  prm.grid = pl.grid;
-  // MMA A operand = weight, B operand = activation.
-  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
-                                kTileN, static_cast<uint32_t>(pl.bn), true);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (pl.bn) {
-    case 16: return launch_linear_bn<16>(dev, 0, tw, ta, prm, st);
-    case 32: return launch_linear_bn<32>(dev, 1, tw, ta, prm, st);
-    case 64: return launch_linear_bn<64>(dev, 2, tw, ta, prm, st);
-    case 128: return launch_linear_bn<128>(dev, 3, tw, ta, prm, st);
-    default: return launch_linear_bn<256>(dev, 4, tw, ta, prm, st);
-  }
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK || empty) return s;
+  const size_t need = pl.partial_bytes + pl.counter_bytes;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+  float* partials = static_cast<float*>(workspace);
+  unsigned int* counters = need > 0 ? reinterpret_cast<unsigned int*>(
+                                          static_cast<uint8_t*>(workspace) + pl.partial_bytes)
+                                    : nullptr;
+  return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                       partials, counters, static_cast<cudaStream_t>(stream));
 }
 
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
@@ -500,26 +559,15 @@ sfp8_status noalloc_scratch(void** out) {
 
 extern "C" sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_dtype,
                                                   const float* s_a, int64_t m,
-                                                  const void* values, const void* meta,
-                                                  sfp8_dtype w_dtype, const float* s_w,
-                                                  int64_t n, int64_t k, const void* bias,
-                                                  void* y, void* stream) {
-  if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
-  if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
-  if (k == 0 || k % kStepK != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 31))
-    return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (m == 0 || n == 0) return SFP8_OK;
-  if (a_q == nullptr || s_a == nullptr || values == nullptr || meta == nullptr ||
-      s_w == nullptr || y == nullptr)
-    return SFP8_ERR_INVALID_ARG;
-  if (!aligned(a_q, 16) || !aligned(values, 16) || !aligned(meta, 16) || !aligned(s_a, 4) ||
-      !aligned(s_w, 4) || !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
-    return SFP8_ERR_MISALIGNED;
+                                                  const void* packed, sfp8_dtype w_dtype,
+                                                  const float* s_w, int64_t n, int64_t k,
+                                                  const void* bias, void* y, void* stream) {
   DeviceInfo* dev = nullptr;
-  sfp8_status s = current_device(&dev);
-  if (s != SFP8_OK) return s;
-  const LinearPlan pl = make_plan(m, n, k, dev->num_sms);
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK || empty) return s;
   if (pl.partial_bytes + pl.counter_bytes > kNoAllocScratchBytes) return SFP8_ERR_WORKSPACE;
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
@@ -528,41 +576,10 @@ extern "C" sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_
   uint8_t* counters = static_cast<uint8_t*>(scratch) + pl.partial_bytes;
   // The buffer keeps whatever the previous call left; the counters must
   // start at zero (the partial sums are always written before being read).
-  if (cudaMemsetAsync(counters, 0, pl.counter_bytes, st) != cudaSuccess) return SFP8_ERR_CUDA;
-
-  CUtensorMap tw, ta;
-  const int64_t n_pad = sfp8_padded_rows(n);
-  s = encode_2d_u8(&tw, values, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n_pad),
-                   static_cast<uint64_t>(k / 2), kStepK / 2, kTileN, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (s != SFP8_OK) return s;
-  s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
-                   static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
-                   CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != SFP8_OK) return s;
-
-  LinearParams prm{};
-  prm.meta = static_cast<const uint8_t*>(meta);
-  prm.s_a = s_a;
-  prm.s_w = s_w;
-  prm.bias = static_cast<const __nv_bfloat16*>(bias);
-  prm.y = static_cast<__nv_bfloat16*>(y);
-  prm.partials = static_cast<float*>(scratch);
-  prm.counters = reinterpret_cast<unsigned int*>(counters);
-  prm.m = static_cast<int>(m);
-  prm.n = static_cast<int>(n);
-  prm.k = static_cast<int>(k);
-  prm.m_tiles = pl.m_tiles;
-  prm.k_steps = pl.k_steps;
-  prm.tiles = pl.tiles;
-  prm.iters = pl.iters;
-  prm.grid = pl.grid;
-  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
-                                kTileN, static_cast<uint32_t>(pl.bn), true);
-  switch (pl.bn) {
-    case 16: return launch_linear_bn<16>(dev, 0, tw, ta, prm, st);
-    case 32: return launch_linear_bn<32>(dev, 1, tw, ta, prm, st);
-    case 64: return launch_linear_bn<64>(dev, 2, tw, ta, prm, st);
-    case 128: return launch_linear_bn<128>(dev, 3, tw, ta, prm, st);
-    default: return launch_linear_bn<256>(dev, 4, tw, ta, prm, st);
-  }
+  if (pl.counter_bytes > 0 &&
+      cudaMemsetAsync(counters, 0, pl.counter_bytes, st) != cudaSuccess)
+    return SFP8_ERR_CUDA;
+  return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                       static_cast<float*>(scratch), reinterpret_cast<unsigned int*>(counters),
+                       st);
 }

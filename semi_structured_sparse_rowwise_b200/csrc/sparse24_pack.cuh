@@ -10,13 +10,18 @@
 // elements beat it, where i beats j when m_i > m_j, or m_i == m_j and i < j
 // (ties to the lower index).
 //
-// Compressed layout (version 1), for an [n, k] weight, n_pad = ceil(n/128)*128:
-//   values [n_pad, k/2] row-major, kept codes group by group (lower index
-//   first); meta in 2048-byte tiles, tile (nt, kt) at (nt*(k/128)+kt)*2048,
-//   row r of the tile at 16*r, byte b = nibbles of groups 2b (bits 0..3) and
-//   2b+1 (bits 4..7) of that 128-wide k tile.  Padding rows: 0x00 values,
-//   nibble 0x4.  Each tile is exactly the 128-lane x 128-bit block that the
-//   GEMM copies into tensor memory for one 128-wide k step of 128 weight rows.
+// Compressed layout (version 3), for an [n, k] weight, n_pad = ceil(n/128)*128:
+// one buffer of 10240-byte tiles, tile t = nt*(k/128) + kt (weight rows
+// 128nt.., k columns 128kt..) at byte 10240*t:
+//   bytes 0..8191: kept values; row r at 64*r holds the row's 64 kept codes
+//   (two per group, lower index first) as four 16-byte chunks, chunk c stored
+//   at position c ^ ((r >> 1) & 3) -- the 64-byte swizzle that the tensor
+//   core's shared-memory descriptor expects.
+//   bytes 8192..10239: index metadata; row r at 8192 + 16*r, byte b = nibbles
+//   of groups 2b (bits 0..3) and 2b+1 (bits 4..7) of the tile's 32 groups --
+//   exactly the 128-lane x 128-bit block the GEMM copies into tensor memory.
+//   Padding rows: 0x00 values, nibble 0x4.
+// A pipeline stage of the GEMM is therefore one contiguous copy.
 #pragma once
 
 #include "device_common.cuh"
@@ -91,7 +96,7 @@ __global__ void prune24_kernel(const Bits* __restrict__ w, int64_t rows, int64_t
 // bytes and 4 metadata bytes.
 __global__ void __launch_bounds__(512)
     compress24_kernel(const uint8_t* __restrict__ wq, int64_t n, int64_t k,
-                      uint8_t* __restrict__ values, uint8_t* __restrict__ meta) {
+                      uint8_t* __restrict__ packed) {
   const int r = threadIdx.x / 4;   // row inside the tile
   const int j = threadIdx.x % 4;   // 32-code chunk inside the 128-wide k tile
   const int64_t kt = blockIdx.x;
@@ -125,15 +130,16 @@ __global__ void __launch_bounds__(512)
     vout[0] = vout[1] = vout[2] = vout[3] = 0;
     mout = 0x44444444u;   // indices (0, 1) in every group
   }
-  *reinterpret_cast<uint4*>(values + row * (k / 2) + kt * 64 + 16 * j) =
+  uint8_t* tile = packed + (nt * ktiles + kt) * 10240;
+  *reinterpret_cast<uint4*>(tile + 64 * r + 16 * (j ^ ((r >> 1) & 3))) =
       make_uint4(vout[0], vout[1], vout[2], vout[3]);
-  *reinterpret_cast<uint32_t*>(meta + (nt * ktiles + kt) * 2048 + 16 * r + 4 * j) = mout;
+  *reinterpret_cast<uint32_t*>(tile + 8192 + 16 * r + 4 * j) = mout;
 }
 
 // Inverse: same thread mapping, n real rows only.
 __global__ void __launch_bounds__(512)
-    decompress24_kernel(const uint8_t* __restrict__ values, const uint8_t* __restrict__ meta,
-                        int64_t n, int64_t k, uint8_t* __restrict__ wq) {
+    decompress24_kernel(const uint8_t* __restrict__ packed, int64_t n, int64_t k,
+                        uint8_t* __restrict__ wq) {
   const int r = threadIdx.x / 4;
   const int j = threadIdx.x % 4;
   const int64_t kt = blockIdx.x;
@@ -141,9 +147,9 @@ __global__ void __launch_bounds__(512)
   const int64_t row = nt * 128 + r;
   if (row >= n) return;
   const int64_t ktiles = k / 128;
-  const uint4 vv = *reinterpret_cast<const uint4*>(values + row * (k / 2) + kt * 64 + 16 * j);
-  const uint32_t mm =
-      *reinterpret_cast<const uint32_t*>(meta + (nt * ktiles + kt) * 2048 + 16 * r + 4 * j);
+  const uint8_t* tile = packed + (nt * ktiles + kt) * 10240;
+  const uint4 vv = *reinterpret_cast<const uint4*>(tile + 64 * r + 16 * (j ^ ((r >> 1) & 3)));
+  const uint32_t mm = *reinterpret_cast<const uint32_t*>(tile + 8192 + 16 * r + 4 * j);
   const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
   uint32_t out[8];
   bool bad = false;

@@ -15,25 +15,31 @@
 // = token m, so in the epilogue the 32 lanes of a warp hold 32 consecutive
 // n of one token and store a contiguous run of y.
 //
-// Structure (one CTA per SM, persistent):
-//   warp 0      TMA producer: per 128-wide k step, the compressed weight tile
-//               (128 x 64 B, 64B swizzle), its 2 KB metadata tile (bulk copy)
-//               and the activation tile (BN x 128 B, 128B swizzle) into one
-//               stage of a multi-stage shared-memory ring.
-//   warp 1      MMA issuer: copies the metadata tile into tensor memory
-//               (tcgen05.cp 128x128b) and issues two 128 x BN x 64 sparse
-//               MMAs per stage; frees the stage with tcgen05.commit.
+// Structure (one or two CTAs per SM, persistent):
+//   warp 0      producer: per stage of KS 128-wide k steps, ONE contiguous
+//               bulk copy of KS packed weight tiles (each 8 KB of kept values,
+//               stored pre-swizzled in the 64B-swizzle form the MMA reads,
+//               followed by its 2 KB of index metadata), and KS TMA copies of
+//               the activation tile (BN x 128 B, 128B swizzle).
+//   warp 1      MMA issuer: per k step, copies the metadata block into tensor
+//               memory (tcgen05.cp 128x128b) and issues two 128 x BN x 64
+//               sparse MMAs; frees the stage with tcgen05.commit.
 //   warps 2-5   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
 //               global, or split-K partials to the workspace.
-// Work split: the (tile, k step) iterations are divided evenly over the
-// CTAs (stream-K).  A CTA whose range covers a tile's whole K finishes it
-// directly; otherwise each part writes an fp32 partial and the last part to
-// arrive (a per-tile counter) adds all parts in a fixed order and finishes
-// the tile, so results do not depend on arrival order.
+// Work split, chosen by the host:
+//   whole tiles  CTA c takes tiles c, c + grid, ...: no partial sums.
+//   stream-K     the (tile, stage) iterations are divided evenly over the
+//                CTAs.  A tile split between CTAs is finished by its last
+//                part: if every other part has already published its fp32
+//                partial (a counter read with acquire semantics), straight
+//                from its registers; otherwise it publishes its own and the
+//                release/acquire counter update picks the finisher.  Parts
+//                are always added in CTA order, so results are bit-identical
+//                run to run whichever part finishes.
 //
 // Every wait is bounded (device_common.cuh): on a timeout the CTA records
-// SFP8_DEVICE_TIMEOUT, lets its copies in flight land, frees its tensor
-// memory and returns.
+// SFP8_DEVICE_TIMEOUT, lets its copies in flight land, drains its MMAs,
+// frees its tensor memory and returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,9 +49,10 @@
 namespace sfp8 {
 
 constexpr int kTileN = 128;     // weight rows per tile (MMA M)
-constexpr int kStepK = 128;     // logical k per pipeline stage
-constexpr int kMetaTileBytes = kTileN * kStepK / 8;   // 2048
-constexpr int kWTileBytes = kTileN * kStepK / 2;      // 8192
+constexpr int kStepK = 128;     // logical k per k step
+constexpr int kWValBytes = kTileN * kStepK / 2;       // 8192: kept values of a tile
+constexpr int kWMetaBytes = kTileN * kStepK / 8;      // 2048: index metadata of a tile
+constexpr int kWTileBytes = kWValBytes + kWMetaBytes;  // 10240: packed tile
 constexpr int kGemmThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kSmemBudget = 225 * 1024;
@@ -56,19 +63,24 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int BN>
+template <int BN, int KS>
 struct LinearCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be 16..256, multiple of 16");
-  static constexpr int kATileBytes = BN * kStepK;
-  static constexpr int kStageBytes = kWTileBytes + kMetaTileBytes + kATileBytes;
-  static constexpr int kNumAcc = (2 * BN + 4 <= 512) ? 2 : 1;
+  static_assert(KS == 1 || KS == 2, "1 or 2 k steps per stage");
+  static constexpr int kATileBytes = BN * kStepK;                 // one k step of activation
+  static constexpr int kStageBytes = KS * (kWTileBytes + kATileBytes);
+  static constexpr int kNumAcc = (2 * BN + 4 * KS <= 512) ? 2 : 1;
   static constexpr int kMetaCol = kNumAcc * BN;
-  static constexpr int kTmemCols = pow2_at_least(kNumAcc * BN + 4);
+  static constexpr int kTmemCols = pow2_at_least(kNumAcc * BN + 4 * KS);
   static constexpr int kBarrierBytes = 1024;
   static constexpr int kStagesMax = 16;
+  // Decode-sized tiles (BN <= 32) use at most half of the SM's shared memory,
+  // so that the next call's CTA can start on the same SM (and stream its
+  // weight) while this one finishes.
+  static constexpr int kBudget = BN <= 32 ? kSmemBudget / 2 - 10 * 1024 : kSmemBudget;
   static constexpr int kStages =
-      ((kSmemBudget - kBarrierBytes - 1024) / kStageBytes) < kStagesMax
-          ? ((kSmemBudget - kBarrierBytes - 1024) / kStageBytes)
+      ((kBudget - kBarrierBytes - 1024) / kStageBytes) < kStagesMax
+          ? ((kBudget - kBarrierBytes - 1024) / kStageBytes)
           : kStagesMax;
   static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kBarrierBytes;
   static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
@@ -76,76 +88,100 @@ struct LinearCfg {
 };
 
 struct LinearParams {
-  const uint8_t* meta;
+  const uint8_t* packed;    // compressed weight, 10 KB tiles (layout version 3)
   const float* s_a;
   const float* s_w;
   const __nv_bfloat16* bias;
   __nv_bfloat16* y;
-  float* partials;          // [grid][2][BN][128] fp32
-  unsigned int* counters;   // [tiles][4]: one per tile and lane quadrant
+  float* partials;          // [grid][2][BN][128] fp32 (stream-K only)
+  unsigned int* counters;   // [tiles][4]: one per tile and lane quadrant (stream-K only)
   int m, n, k;
   int m_tiles;              // ceil(m / BN)
   int k_steps;              // k / 128
+  int units;                // stages per tile: k_steps / KS
   long long tiles;          // n_tiles * m_tiles
-  long long iters;          // tiles * k_steps
+  long long iters;          // tiles * units
   int grid;
+  int whole_tiles;          // 1: CTA c takes tiles c, c + grid, ...; 0: stream-K
   uint32_t idesc;
 };
 
-// The contiguous range of (tile, k step) iterations owned by a CTA, walked
-// one tile segment at a time.  All three roles walk it identically.
+// The work of one CTA, one tile segment [u0, u1) (in stages) at a time.  All
+// three roles walk it identically.
 struct SegmentWalker {
   long long it, end;
-  int k_steps;
+  int units;
+  int grid;
+  bool whole;
   __device__ SegmentWalker(const LinearParams& p, int cta) {
-    it = static_cast<long long>(cta) * p.iters / p.grid;
-    end = static_cast<long long>(cta + 1) * p.iters / p.grid;
-    k_steps = p.k_steps;
+    units = p.units;
+    grid = p.grid;
+    whole = p.whole_tiles != 0;
+    if (whole) {
+      it = cta;               // next tile
+      end = p.tiles;
+    } else {
+      it = static_cast<long long>(cta) * p.iters / p.grid;
+      end = static_cast<long long>(cta + 1) * p.iters / p.grid;
+    }
   }
-  __device__ bool next(long long& tile, int& kb0, int& kb1) {
+  __device__ bool next(long long& tile, int& u0, int& u1) {
     if (it >= end) return false;
-    tile = it / k_steps;
-    kb0 = static_cast<int>(it % k_steps);
+    if (whole) {
+      tile = it;
+      u0 = 0;
+      u1 = units;
+      it += grid;
+      return true;
+    }
+    tile = it / units;
+    u0 = static_cast<int>(it % units);
     const long long left = end - it;
-    kb1 = static_cast<int>(left < k_steps - kb0 ? kb0 + left : k_steps);
-    it += kb1 - kb0;
+    u1 = static_cast<int>(left < units - u0 ? u0 + left : units);
+    it += u1 - u0;
     return true;
   }
 };
 
-// CTA owning iteration i (the inverse of the even split).
+// Stream-K: CTA owning iteration i (the inverse of the even split).
 __device__ __forceinline__ int cta_of_iter(long long i, const LinearParams& p) {
   return static_cast<int>(((i + 1) * p.grid - 1) / p.iters);
 }
 
+// Stream-K: partial-sum slot of CTA `cc` for `tile`: slot 0 holds the part of
+// the tile its range starts in, slot 1 the part of the tile its range ends in.
 template <int BN>
-__device__ __forceinline__ void tile_coords(const LinearParams& p, long long tile, int& nt,
-                                            int& mt) {
-  nt = static_cast<int>(tile / p.m_tiles);
-  mt = static_cast<int>(tile % p.m_tiles);
+__device__ __forceinline__ const float* partial_slot(const LinearParams& p, int cc,
+                                                     long long tile) {
+  const long long start = static_cast<long long>(cc) * p.iters / p.grid;
+  const int slot = (start / p.units == tile) ? 0 : 1;
+  return p.partials + (static_cast<long long>(cc) * 2 + slot) * (BN * kTileN);
 }
 
-// Epilogue for one 16-column chunk held in registers: y = acc*s_a*s_w + bias.
-template <int BN>
+// Epilogue of one 16-column chunk: y = acc * (s_a * s_w) + bias.
 __device__ __forceinline__ void store_chunk(const LinearParams& p, const float (&acc)[16],
-                                            int n, int m0, float sw, float bias) {
+                                            const float (&sa)[16], int n, int m0, float sw,
+                                            float bias) {
   if (n >= p.n) return;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int m = m0 + j;
     if (m < p.m) {
-      const float sa = __ldg(p.s_a + m);
-      const float v = fmaf(acc[j], sa * sw, bias);
+      const float v = fmaf(acc[j], sa[j] * sw, bias);
       p.y[static_cast<long long>(m) * p.n + n] = __float2bfloat16_rn(v);
     }
   }
 }
 
-template <int BN>
+__device__ __forceinline__ void load_sa(const LinearParams& p, int m0, float (&sa)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) sa[j] = (m0 + j < p.m) ? __ldg(p.s_a + m0 + j) : 0.0f;
+}
+
+template <int BN, int KS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_w,
-                         const __grid_constant__ CUtensorMap tm_a, const LinearParams p) {
-  using Cfg = LinearCfg<BN>;
+    sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_a, const LinearParams p) {
+  using Cfg = LinearCfg<BN, KS>;
   constexpr int S = Cfg::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -163,6 +199,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int cta = blockIdx.x;
+  // Dependent kernels of this library may launch right away: each of them
+  // waits (griddepcontrol.wait) for this grid to complete before it reads or
+  // writes anything this grid uses, so an early trigger only lets their
+  // launch and their own weight prefetch overlap this grid's tail.
+  grid_dependents_launch();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -177,10 +218,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_a);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_a);
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     tmem_relinquish();
@@ -193,59 +231,60 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
+      // A weight tile is read once when there is one token tile (decode:
+      // keep it from displacing anything); otherwise every token tile reuses
+      // it, so it must stay in L2.
+      const uint64_t pol_w = p.m_tiles == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
       const uint64_t pol_a = l2_policy_evict_last();
+      auto issue_weight = [&](int stage, long long tile, int u) {
+        const int nt = static_cast<int>(tile / p.m_tiles);
+        uint8_t* st = stage_base + stage * Cfg::kStageBytes;
+        const uint32_t fb = smem_u32(&full_bar[stage]);
+        mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+        bulk_load(smem_u32(st),
+                  p.packed + (static_cast<long long>(nt) * p.k_steps + u * KS) * kWTileBytes,
+                  KS * kWTileBytes, fb, pol_w);
+      };
+      auto issue_act = [&](int stage, long long tile, int u) {
+        const int mt = static_cast<int>(tile % p.m_tiles);
+        uint8_t* st = stage_base + stage * Cfg::kStageBytes + KS * kWTileBytes;
+        const uint32_t fb = smem_u32(&full_bar[stage]);
+#pragma unroll
+        for (int j = 0; j < KS; ++j)
+          tma_load_2d(smem_u32(st + j * Cfg::kATileBytes), &tm_a, (u * KS + j) * kStepK,
+                      mt * BN, fb, pol_a);
+      };
+      // The weight does not depend on the preceding kernel: fill the first
+      // stages with weight tiles before waiting for the activation.
+      long long pre_count = 0;
+      {
+        SegmentWalker pre(p, cta);
+        long long t2;
+        int a0, a1;
+        while (pre_count < S && pre.next(t2, a0, a1))
+          for (int u = a0; u < a1 && pre_count < S; ++u) {
+            issue_weight(static_cast<int>(pre_count), t2, u);
+            ++pre_count;
+          }
+      }
+      grid_dependency_wait();
       SegmentWalker walk(p, cta);
       long long tile;
-      int kb0, kb1;
+      int u0, u1;
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
-      // The weight does not depend on the preceding kernel: fill the first
-      // stages with weight tiles before waiting for the activation.
-      SegmentWalker pre(p, cta);
-      int pre_stage = 0;
-      long long pre_count = 0;
-      {
-        long long t2;
-        int a0, a1;
-        while (pre_count < S && pre.next(t2, a0, a1)) {
-          int nt, mt;
-          tile_coords<BN>(p, t2, nt, mt);
-          for (int kb = a0; kb < a1 && pre_count < S; ++kb) {
-            uint8_t* st = stage_base + pre_stage * Cfg::kStageBytes;
-            const uint32_t fb = smem_u32(&full_bar[pre_stage]);
-            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-            tma_load_2d(smem_u32(st), &tm_w, kb * (kStepK / 2), nt * kTileN, fb, pol_w);
-            bulk_load(smem_u32(st + kWTileBytes),
-                      p.meta + (static_cast<long long>(nt) * p.k_steps + kb) * kMetaTileBytes,
-                      kMetaTileBytes, fb, pol_w);
-            ++pre_stage;
-            ++pre_count;
-          }
-        }
-      }
-      grid_dependency_wait();
       bool ok = true;
-      while (ok && walk.next(tile, kb0, kb1)) {
-        int nt, mt;
-        tile_coords<BN>(p, tile, nt, mt);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          uint8_t* st = stage_base + stage * Cfg::kStageBytes;
-          const uint32_t fb = smem_u32(&full_bar[stage]);
+      while (ok && walk.next(tile, u0, u1)) {
+        for (int u = u0; u < u1; ++u) {
           if (issued >= pre_count) {
             if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-            tma_load_2d(smem_u32(st), &tm_w, kb * (kStepK / 2), nt * kTileN, fb, pol_w);
-            bulk_load(smem_u32(st + kWTileBytes),
-                      p.meta + (static_cast<long long>(nt) * p.k_steps + kb) * kMetaTileBytes,
-                      kMetaTileBytes, fb, pol_w);
+            issue_weight(stage, tile, u);
           }
-          tma_load_2d(smem_u32(st + kWTileBytes + kMetaTileBytes), &tm_a, kb * kStepK,
-                      mt * BN, fb, pol_a);
+          issue_act(stage, tile, u);
           ++issued;
           if (++stage == S) {
             stage = 0;
@@ -268,41 +307,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      grid_dependency_wait();   // start the wait limits only once inputs exist
       SegmentWalker walk(p, cta);
       long long tile;
-      int kb0, kb1;
+      int u0, u1;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       const uint32_t e_tmem = tmem_base + Cfg::kMetaCol;
       bool ok = true;
-      while (ok && walk.next(tile, kb0, kb1)) {
+      while (ok && walk.next(tile, u0, u1)) {
         if (!mbar_wait(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int u = u0; u < u1; ++u) {
           if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t st = smem_u32(stage_base + stage * Cfg::kStageBytes);
-          const uint32_t w_addr = st;
-          const uint32_t e_addr = st + kWTileBytes;
-          const uint32_t a_addr = st + kWTileBytes + kMetaTileBytes;
-          // metadata: 128 rows x 16 bytes, no swizzle, 8-row groups 128 B apart
-          tc_cp_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kNoSwizzle));
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            // weight: 128 rows x 64 B (64B swizzle, 8-row atoms 512 B apart);
-            // each MMA consumes 32 B of every row (64 logical k).
-            const uint64_t adesc = smem_desc(w_addr + 32 * j, 16, 512, kSwizzle64);
-            // activation: BN rows x 128 B (128B swizzle, atoms 1024 B apart);
-            // each MMA consumes 64 B of every row.
-            const uint64_t bdesc = smem_desc(a_addr + 64 * j, 16, 1024, kSwizzle128);
-            mma_sp_f8f6f4(d_tmem, adesc, bdesc, e_tmem + 2 * j, p.idesc,
-                          (kb > kb0 || j > 0) ? 1u : 0u);
+          for (int j = 0; j < KS; ++j) {
+            const uint32_t w_addr = st + j * kWTileBytes;
+            const uint32_t e_addr = w_addr + kWValBytes;
+            const uint32_t a_addr = st + KS * kWTileBytes + j * Cfg::kATileBytes;
+            // metadata: 128 rows x 16 bytes, no swizzle, 8-row groups 128 B apart
+            tc_cp_128x128b(e_tmem + 4 * j, smem_desc(e_addr, 0, 128, kNoSwizzle));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // weight: 128 rows x 64 B (64B swizzle, 8-row atoms 512 B apart);
+              // each MMA consumes 32 B of every row (64 logical k).
+              const uint64_t adesc = smem_desc(w_addr + 32 * h, 16, 512, kSwizzle64);
+              // activation: BN rows x 128 B (128B swizzle, atoms 1024 B apart);
+              // each MMA consumes 64 B of every row.
+              const uint64_t bdesc = smem_desc(a_addr + 64 * h, 16, 1024, kSwizzle128);
+              mma_sp_f8f6f4(d_tmem, adesc, bdesc, e_tmem + 4 * j + 2 * h, p.idesc,
+                            (u > u0 || j > 0 || h > 0) ? 1u : 0u);
+            }
           }
           tc_commit(smem_u32(&empty_bar[stage]));
           if (++stage == S) {
@@ -333,24 +376,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp % 4;
     SegmentWalker walk(p, cta);
     long long tile;
-    int kb0, kb1;
+    int u0, u1;
     int acc = 0;
     uint32_t acc_phase = 0;
     long long first_tile = -1;
-    while (walk.next(tile, kb0, kb1)) {
+    while (walk.next(tile, u0, u1)) {
       if (first_tile < 0) first_tile = tile;
+      const int nt = static_cast<int>(tile / p.m_tiles);
+      const int mt = static_cast<int>(tile % p.m_tiles);
+      const int n_local = q * 32 + lane;
+      const int n = nt * kTileN + n_local;
+      const bool whole = (u0 == 0 && u1 == p.units);
+      // Everything the epilogue needs besides the accumulator, loaded before
+      // waiting for it.
+      const float sw = (n < p.n) ? __ldg(p.s_w + n) : 0.0f;
+      const float bv = (p.bias != nullptr && n < p.n) ? __bfloat162float(p.bias[n]) : 0.0f;
+      float sa0[16];
+      load_sa(p, mt * BN, sa0);
+      int c_first = cta, c_last = cta;
+      unsigned int parts = 1;
+      unsigned int* counter = p.counters + tile * 4 + q;
+      if (!whole) {
+        const long long it0 = tile * p.units;
+        c_first = cta_of_iter(it0, p);
+        c_last = cta_of_iter(it0 + p.units - 1, p);
+        parts = static_cast<unsigned int>(c_last - c_first + 1);
+      }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(smem_u32(&accf_bar[acc]), acc_phase, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
+      // Split tile: finish it here if every other part has already arrived.
+      bool finish_now = false;
+      if (!whole) {
+        unsigned int arrived = 0;
+        if (lane == 0) arrived = load_acquire_gpu(counter);
+        finish_now = __shfl_sync(0xffffffffu, arrived, 0) + 1 == parts;
+      }
       tc_fence_after();
-      int nt, mt;
-      tile_coords<BN>(p, tile, nt, mt);
-      const int n_local = q * 32 + lane;
-      const int n = nt * kTileN + n_local;
-      const bool whole = (kb0 == 0 && kb1 == p.k_steps);
-      const float sw = (n < p.n) ? __ldg(p.s_w + n) : 0.0f;
-      const float bv = (p.bias != nullptr && n < p.n) ? __bfloat162float(p.bias[n]) : 0.0f;
       const int slot = (tile == first_tile) ? 0 : 1;
       float* part = p.partials + (static_cast<long long>(cta) * 2 + slot) * (BN * kTileN);
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
@@ -358,12 +421,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int c = 0; c < BN / 16; ++c) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(t_row + c * 16, r);
+        float sa[16];
+        if (c == 0) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sa[j] = sa0[j];
+        } else {
+          load_sa(p, mt * BN + c * 16, sa);
+        }
         tmem_ld_wait();
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
         if (whole) {
-          store_chunk<BN>(p, v, n, mt * BN + c * 16, sw, bv);
+          store_chunk(p, v, sa, n, mt * BN + c * 16, sw, bv);
+        } else if (finish_now) {
+          float sum[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sum[j] = 0.0f;
+          for (int cc = c_first; cc <= c_last; ++cc) {
+            if (cc == cta) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sum[j] += v[j];
+            } else {
+              const float* src = partial_slot<BN>(p, cc, tile) + c * 16 * kTileN + n_local;
+              float a[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) a[j] = __ldcg(src + j * kTileN);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) sum[j] += a[j];
+            }
+          }
+          store_chunk(p, sum, sa, n, mt * BN + c * 16, sw, bv);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) part[(c * 16 + j) * kTileN + n_local] = v[j];
@@ -378,39 +466,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else {
         acc_phase ^= 1u;
       }
-      if (!whole) {
-        // Publish this warp's part of the split tile; the last part to
-        // arrive (per tile and quadrant) adds all parts in CTA order.
-        __threadfence();
+      if (finish_now) {
+        if (lane == 0) *counter = 0u;   // every other part has counted already
+      } else if (!whole) {
+        // The counter update is a release/acquire atomic: it orders this
+        // warp's part (stores ordered across the warp by __syncwarp) before
+        // the count and, for the last part, every other part before the
+        // loads below.
         __syncwarp();
-        const long long it0 = tile * p.k_steps;
-        const int c_first = cta_of_iter(it0, p);
-        const int c_last = cta_of_iter(it0 + p.k_steps - 1, p);
         unsigned int last = 0;
-        if (lane == 0) {
-          const unsigned int parts = static_cast<unsigned int>(c_last - c_first + 1);
-          const unsigned int prev = atomicAdd(p.counters + tile * 4 + q, 1u);
-          last = (prev + 1 == parts) ? 1u : 0u;
-        }
+        if (lane == 0) last = (atomic_add_acq_rel_gpu(counter, 1u) + 1 == parts) ? 1u : 0u;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (last) {
-          __threadfence();
+          __syncwarp();
 #pragma unroll 1
           for (int c = 0; c < BN / 16; ++c) {
+            float sa[16];
+            load_sa(p, mt * BN + c * 16, sa);
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-            for (int cc = c_first; cc <= c_last; ++cc) {
-              const long long cc_start = static_cast<long long>(cc) * p.iters / p.grid;
-              const int cc_slot = (cc_start / p.k_steps == tile) ? 0 : 1;
-              const float* src =
-                  p.partials + (static_cast<long long>(cc) * 2 + cc_slot) * (BN * kTileN);
+            int cc = c_first;
+            // two parts per round trip; additions stay in CTA order
+            for (; cc + 1 <= c_last; cc += 2) {
+              const float* s0 = partial_slot<BN>(p, cc, tile) + c * 16 * kTileN + n_local;
+              const float* s1 = partial_slot<BN>(p, cc + 1, tile) + c * 16 * kTileN + n_local;
+              float a0[16], a1[16];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) v[j] += __ldcg(src + (c * 16 + j) * kTileN + n_local);
+              for (int j = 0; j < 16; ++j) {
+                a0[j] = __ldcg(s0 + j * kTileN);
+                a1[j] = __ldcg(s1 + j * kTileN);
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] = (v[j] + a0[j]) + a1[j];
             }
-            store_chunk<BN>(p, v, n, mt * BN + c * 16, sw, bv);
+            if (cc <= c_last) {
+              const float* s0 = partial_slot<BN>(p, cc, tile) + c * 16 * kTileN + n_local;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) v[j] += __ldcg(s0 + j * kTileN);
+            }
+            store_chunk(p, v, sa, n, mt * BN + c * 16, sw, bv);
           }
-          if (lane == 0) p.counters[tile * 4 + q] = 0u;
+          if (lane == 0) *counter = 0u;
         }
       }
     }

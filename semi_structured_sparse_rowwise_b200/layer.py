@@ -25,19 +25,18 @@ class SparseFp8Linear:
         self.device = weight.device
         w = B.sfp8_prune_24(weight.contiguous()) if prune else weight.contiguous()
         w_q, self.s_w = B.sfp8_quantize_rowwise(w, w_dtype)
-        self.values, self.meta = B.sfp8_compress_24(w_q, w_dtype)
+        self.packed = B.sfp8_compress_24(w_q, w_dtype)
         self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
         self._ws = {}
 
     @classmethod
-    def from_compressed(cls, values, meta, s_w, n, k, bias=None, w_dtype="e4m3",
-                        a_dtype="e4m3"):
-        """A layer over an already compressed weight (values, meta, s_w)."""
+    def from_compressed(cls, packed, s_w, n, k, bias=None, w_dtype="e4m3", a_dtype="e4m3"):
+        """A layer over an already compressed weight (packed, s_w)."""
         self = cls.__new__(cls)
         self.n, self.k = n, k
         self.w_dtype, self.a_dtype = w_dtype, a_dtype
-        self.device = values.device
-        self.values, self.meta, self.s_w = values, meta, s_w
+        self.device = packed.device
+        self.packed, self.s_w = packed, s_w
         self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
         self._ws = {}
         return self
@@ -52,7 +51,7 @@ class SparseFp8Linear:
     def forward(self, x, out=None):
         """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16."""
         a_q, s_a = B.sfp8_quantize_rowwise(x, self.a_dtype)
-        return B.sfp8_sparse_linear(a_q, self.a_dtype, s_a, self.values, self.meta,
+        return B.sfp8_sparse_linear(a_q, self.a_dtype, s_a, self.packed,
                                     self.w_dtype, self.s_w, self.n, self.k, bias=self.bias,
                                     out=out, workspace=self.workspace(x.shape[0]))
 

@@ -44,13 +44,13 @@ class GpuLayer:
         self.w = bf16_dev(w_bits)
         self.wp = S.sfp8_prune_24(self.w)
         self.wq, self.sw = S.sfp8_quantize_rowwise(self.wp, w_fmt)
-        self.values, self.meta = S.sfp8_compress_24(self.wq, w_fmt)
+        self.packed = S.sfp8_compress_24(self.wq, w_fmt)
 
     def forward(self, x_bits, a_fmt, bias_bits=None):
         x = bf16_dev(x_bits)
         aq, sa = S.sfp8_quantize_rowwise(x, a_fmt)
         bias = bf16_dev(bias_bits) if bias_bits is not None else None
-        y = S.sfp8_sparse_linear(aq, a_fmt, sa, self.values, self.meta, self.w_fmt, self.sw,
+        y = S.sfp8_sparse_linear(aq, a_fmt, sa, self.packed, self.w_fmt, self.sw,
                                  self.n, self.k, bias=bias)
         return aq, sa, y
 
@@ -97,8 +97,8 @@ def check_weight_prep(gl, rl, cols):
     assert np.array_equal(wq, rl.wq), "quantised weight codes differ"
     sw = gl.sw.index_select(0, cols_t).cpu().numpy()
     assert np.array_equal(sw.view(np.uint32), rl.sw.view(np.uint32)), "weight scales differ"
-    vals, nib = oracle.unpack_physical(gl.values.cpu().numpy(), gl.meta.cpu().numpy(), gl.n,
-                                       gl.k, include_padding=True)
+    vals, nib = oracle.unpack_physical(gl.packed.cpu().numpy(), gl.n, gl.k,
+                                       include_padding=True)
     assert np.array_equal(vals[cols], rl.vals), "kept values differ"
     assert np.array_equal(nib[cols], rl.nib), "index nibbles differ"
     npad = vals.shape[0]

@@ -43,12 +43,11 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_layout_constants_match(lib):
-    assert lib.sfp8_layout_version() == 1 == oracle.layout.LAYOUT_VERSION
+    assert lib.sfp8_layout_version() == 3 == oracle.layout.LAYOUT_VERSION
     for n in (0, 1, 127, 128, 129, 14336, 28672):
         assert lib.sfp8_padded_rows(n) == oracle.padded_rows(n)
         for k in (128, 4096, 14336):
-            assert lib.sfp8_compressed_values_bytes(n, k) == oracle.values_bytes(n, k)
-            assert lib.sfp8_compressed_meta_bytes(n, k) == oracle.meta_bytes(n, k)
+            assert lib.sfp8_compressed_bytes(n, k) == oracle.packed_bytes(n, k)
 
 
 def test_status_strings(lib):
@@ -79,21 +78,22 @@ def test_prune_compress_validation_without_gpu(lib):
     assert lib.sfp8_prune_24(FAKE, 3, 4, 16, 16, FAKE, None) == 4
     assert lib.sfp8_prune_24(FAKE, 0, 4, 20, 20, FAKE, None) == 2
     assert lib.sfp8_prune_24(FAKE, 0, 4, 16, 32, FAKE, None) == 1   # in place needs ld == cols
-    assert lib.sfp8_compress_24(FAKE, 0, 4, 128, FAKE, FAKE, None) == 4
-    assert lib.sfp8_compress_24(FAKE, 3, 4, 192, FAKE, FAKE, None) == 2
-    assert lib.sfp8_compress_24(FAKE, 3, 4, 0, FAKE, FAKE, None) == 2
-    assert lib.sfp8_compress_24(FAKE, 3, 0, 128, FAKE, FAKE, None) == 0
-    assert lib.sfp8_compress_24(FAKE_ODD, 3, 4, 128, FAKE, FAKE, None) == 3
-    assert lib.sfp8_decompress_24(FAKE, FAKE, 4, 100, FAKE, None) == 2
+    assert lib.sfp8_compress_24(FAKE, 0, 4, 128, FAKE, None) == 4
+    assert lib.sfp8_compress_24(FAKE, 3, 4, 192, FAKE, None) == 2
+    assert lib.sfp8_compress_24(FAKE, 3, 4, 0, FAKE, None) == 2
+    assert lib.sfp8_compress_24(FAKE, 3, 0, 128, FAKE, None) == 0
+    assert lib.sfp8_compress_24(FAKE_ODD, 3, 4, 128, FAKE, None) == 3
+    assert lib.sfp8_compress_24(FAKE, 3, 4, 128, FAKE_ODD, None) == 3
+    assert lib.sfp8_decompress_24(FAKE, 4, 100, FAKE, None) == 2
 
 
 def test_linear_validation_without_gpu(lib):
     f = lib.sfp8_sparse_linear
-    args = [FAKE, 3, FAKE, 16, FAKE, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE, 1 << 20, None]
+    args = [FAKE, 3, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE, 1 << 20, None]
 
     def call(**kw):
         a = list(args)
-        names = ["a_q", "a_dt", "s_a", "m", "vals", "meta", "w_dt", "s_w", "n", "k", "bias",
+        names = ["a_q", "a_dt", "s_a", "m", "packed", "w_dt", "s_w", "n", "k", "bias",
                  "y", "ws", "wsb", "stream"]
         for key, v in kw.items():
             a[names.index(key)] = v
@@ -110,3 +110,8 @@ def test_linear_validation_without_gpu(lib):
     assert call(a_q=FAKE_ODD) == 3
     assert call(bias=FAKE_ODD) == 3
     assert call(s_w=ctypes.c_void_p(0x10002)) == 3
+    assert call(packed=FAKE_ODD) == 3
+    na = lib.sfp8_sparse_linear_noalloc
+    assert na(FAKE, 0, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 4
+    assert na(FAKE, 3, FAKE, 16, FAKE, 3, FAKE, 64, 0, None, FAKE, None) == 2
+    assert na(FAKE, 3, FAKE, 0, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 0

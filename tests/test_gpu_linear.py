@@ -72,14 +72,13 @@ def test_deterministic_and_counters_reset():
     xd = bf16_dev(x)
     aq, sa = S.sfp8_quantize_rowwise(xd, "e4m3")
     ws = S.new_workspace(m, n, k, xd.device)
-    y1 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.values, gl.meta, "e4m3", gl.sw, n, k,
-                              workspace=ws)
-    y2 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.values, gl.meta, "e4m3", gl.sw, n, k,
-                              workspace=ws)
+    y1 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.packed, "e4m3", gl.sw, n, k, workspace=ws)
+    y2 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.packed, "e4m3", gl.sw, n, k, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     nbytes = S.sfp8_sparse_linear_workspace_bytes(m, n, k)
     tiles = ((n + 127) // 128) * 1
+    assert nbytes >= tiles * 16           # this shape is split across CTAs
     counters = ws[nbytes - tiles * 16: nbytes].view(torch.int32)
     assert int(counters.abs().sum()) == 0
     _status_clean()
@@ -87,12 +86,12 @@ def test_deterministic_and_counters_reset():
 
 def test_workspace_too_small():
     m, k, n = 16, 256, 256
+    assert S.sfp8_sparse_linear_workspace_bytes(m, n, k) > 16     # split-K shape
     gl = GpuLayer(synthetic.weight(3, n, k), "e4m3")
     aq, sa = S.sfp8_quantize_rowwise(bf16_dev(synthetic.activation(4, m, k)), "e4m3")
     small = torch.zeros((16,), dtype=torch.uint8, device="cuda")
     with pytest.raises(S.Sfp8Error) as e:
-        S.sfp8_sparse_linear(aq, "e4m3", sa, gl.values, gl.meta, "e4m3", gl.sw, n, k,
-                             workspace=small)
+        S.sfp8_sparse_linear(aq, "e4m3", sa, gl.packed, "e4m3", gl.sw, n, k, workspace=small)
     assert e.value.status == 6
 
 

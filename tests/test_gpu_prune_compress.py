@@ -52,11 +52,11 @@ def test_compress_brute_force_groups():
     groups = np.array(list(itertools.product(codes, repeat=4)), dtype=np.uint8)   # 20736 x 4
     q = groups.reshape(-1, 128)                                                   # 648 rows
     n, k = q.shape
-    vals_d, meta_d = S.sfp8_compress_24(torch.from_numpy(q).cuda(), "e4m3")
-    vals, nib = oracle.unpack_physical(vals_d.cpu().numpy(), meta_d.cpu().numpy(), n, k)
+    packed = S.sfp8_compress_24(torch.from_numpy(q).cuda(), "e4m3")
+    vals, nib = oracle.unpack_physical(packed.cpu().numpy(), n, k)
     vr, nr = oracle.compress_24(q, "e4m3")
     assert np.array_equal(vals, vr) and np.array_equal(nib, nr)
-    back = S.sfp8_decompress_24(vals_d, meta_d, n, k).cpu().numpy()
+    back = S.sfp8_decompress_24(packed, n, k).cpu().numpy()
     assert np.array_equal(back, oracle.decompress_24(vr, nr, k))
     _device_status_clean()
 
@@ -64,9 +64,9 @@ def test_compress_brute_force_groups():
 def test_compress_idempotent_on_gpu():
     w_bits = synthetic.weight(5, 256, 512, neg_zero_frac=0.05)
     gl = GpuLayer(w_bits, "e4m3")
-    back = S.sfp8_decompress_24(gl.values, gl.meta, 256, 512)
-    v2, m2 = S.sfp8_compress_24(back, "e4m3")
-    assert torch.equal(v2, gl.values) and torch.equal(m2, gl.meta)
+    back = S.sfp8_decompress_24(gl.packed, 256, 512)
+    p2 = S.sfp8_compress_24(back, "e4m3")
+    assert torch.equal(p2, gl.packed)
 
 
 def test_stress_weight_sampled():

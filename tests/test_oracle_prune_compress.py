@@ -108,25 +108,29 @@ def test_pipeline_invariants(fmt):
 
 
 def test_layout_unpacker_against_loop_packer():
-    """Pack by explicit loops from the layout's byte formulas, then unpack."""
+    """Pack by explicit loops from the layout's byte formula, then unpack."""
     n, k = 130, 256
     rng = np.random.Generator(np.random.PCG64(9))
     vals = rng.integers(0, 256, (n, k // 2), dtype=np.uint8)
     nib = rng.choice(np.array(oracle.NIBBLES_VALID, dtype=np.uint8), (n, k // 4))
     npad = oracle.padded_rows(n)
     assert npad == 256
-    vphys = np.zeros(npad * k // 2, dtype=np.uint8)
-    mphys = np.zeros(npad * k // 8, dtype=np.uint8)
+    phys = np.zeros(npad * k * 5 // 8, dtype=np.uint8)
+    assert phys.size == oracle.packed_bytes(n, k)
     for row in range(npad):
+        nt, r = divmod(row, 128)
         for j in range(k // 2):
-            vphys[row * (k // 2) + j] = vals[row, j] if row < n else 0
+            kt, jj = divmod(j, 64)          # 64 value bytes per 128-wide K step
+            c, b = divmod(jj, 16)           # 16-byte chunk c, byte b
+            pos = c ^ ((r >> 1) & 3)
+            byte = (nt * (k // 128) + kt) * 10240 + 64 * r + 16 * pos + b
+            phys[byte] = vals[row, j] if row < n else 0
         for grp in range(k // 4):
             v = nib[row, grp] if row < n else 0x4
-            nt, r = divmod(row, 128)
             kt, gg = divmod(grp, 32)
-            byte = (nt * (k // 128) + kt) * 2048 + 16 * r + gg // 2
-            mphys[byte] |= v << (4 * (gg % 2))
-    v_out, n_out = oracle.unpack_physical(vphys, mphys, n, k)
+            byte = (nt * (k // 128) + kt) * 10240 + 8192 + 16 * r + gg // 2
+            phys[byte] |= v << (4 * (gg % 2))
+    v_out, n_out = oracle.unpack_physical(phys, n, k)
     assert np.array_equal(v_out, vals) and np.array_equal(n_out, nib)
-    v_all, n_all = oracle.unpack_physical(vphys, mphys, n, k, include_padding=True)
+    v_all, n_all = oracle.unpack_physical(phys, n, k, include_padding=True)
     assert np.all(v_all[n:] == 0) and np.all(n_all[n:] == 0x4)

@@ -42,8 +42,7 @@ def test_noalloc_matches_workspace_entry_point(m, k, n, a_fmt, w_fmt, with_bias)
     gl = GpuLayer(w, w_fmt)
     aq, sa = S.sfp8_quantize_rowwise(bf16_dev(x), a_fmt)
     bias = bf16_dev(b) if b is not None else None
-    y_ws = S.sfp8_sparse_linear(aq, a_fmt, sa, gl.values, gl.meta, w_fmt, gl.sw, n, k,
-                                bias=bias)
+    y_ws = S.sfp8_sparse_linear(aq, a_fmt, sa, gl.packed, w_fmt, gl.sw, n, k, bias=bias)
     # the acceptance bound's terms, from the oracle on the same inputs
     rl = RefLayer(w, w_fmt)
     _, aq_r, sa_r = rl.act(x, a_fmt)
@@ -51,7 +50,7 @@ def test_noalloc_matches_workspace_entry_point(m, k, n, a_fmt, w_fmt, with_bias)
     ref = y_ws.float().cpu().numpy().astype(np.float64)
     for _ in range(2):
         out = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
-        y_na = S.sfp8_sparse_linear_noalloc(aq, a_fmt, sa, gl.values, gl.meta, w_fmt, gl.sw,
+        y_na = S.sfp8_sparse_linear_noalloc(aq, a_fmt, sa, gl.packed, w_fmt, gl.sw,
                                             n, k, bias=bias, out=out)
         torch.cuda.synchronize()
         got = y_na.float().cpu().numpy().astype(np.float64)
@@ -68,9 +67,8 @@ def test_noalloc_rejects_problems_beyond_its_buffer():
     assert S.sfp8_sparse_linear_workspace_bytes(m, n, k) > 8 << 20
     aq = torch.zeros((m, k), dtype=torch.uint8, device="cuda")
     sa = torch.ones((m,), dtype=torch.float32, device="cuda")
-    vals = torch.zeros((S.sfp8_compressed_values_bytes(n, k),), dtype=torch.uint8, device="cuda")
-    meta = torch.zeros((S.sfp8_compressed_meta_bytes(n, k),), dtype=torch.uint8, device="cuda")
+    packed = torch.zeros((S.sfp8_compressed_bytes(n, k),), dtype=torch.uint8, device="cuda")
     sw = torch.ones((n,), dtype=torch.float32, device="cuda")
     with pytest.raises(S.Sfp8Error) as e:
-        S.sfp8_sparse_linear_noalloc(aq, "e4m3", sa, vals, meta, "e4m3", sw, n, k)
+        S.sfp8_sparse_linear_noalloc(aq, "e4m3", sa, packed, "e4m3", sw, n, k)
     assert e.value.status == 6      # SFP8_ERR_WORKSPACE
