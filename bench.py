@@ -72,9 +72,20 @@ def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+        return float(d["hbm_gbs"]), "measured hbm_gbs (MEASURED_PEAKS.json)"
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, "fallback 6.65 TB/s"
+
+
+def measured_tensor_peak():
+    """Dense-equivalent 2:4 sparse FP8 peak: the measured bf16 burst peak x 2
+    (FP8 vs bf16) x 2 (2:4 sparsity), the nominal B200 ratios."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return 4.0 * float(d["bf16_tflops"]), "4 x measured bf16_tflops burst (MEASURED_PEAKS.json)"
+    except Exception:
+        return 4.0 * 1590.0, "4 x fallback 1.59 PFLOP/s"
 
 
 class ClockSampler:
@@ -261,8 +272,13 @@ def run_ours(args):
     from semi_structured_sparse_rowwise_b200 import synthetic
 
     S.load_library()
-    m = args.m
-    x_bits, w_bits, _, seeds = synthetic.workload_inputs(WORKLOAD, M_TO_SHAPE[m])
+    prefill = args.workload == "prefill_8b"
+    if prefill:
+        x_bits, w_bits, _, seeds = synthetic.workload_inputs("prefill_8b", args.shape)
+        m = x_bits.shape[0]
+    else:
+        m = args.m
+        x_bits, w_bits, _, seeds = synthetic.workload_inputs(WORKLOAD, M_TO_SHAPE[m])
     n, k = w_bits.shape
     stream = torch.cuda.current_stream(dev)
 
@@ -306,19 +322,22 @@ def run_ours(args):
     }
 
     # ---- the step's buffers
-    copies = [(packed.clone(), sw.clone()) for _ in range(WEIGHT_COPIES)]
+    n_copies = WEIGHT_COPIES if not prefill else max(
+        2, -(-150 * 2 ** 20 // (packed.numel() + m * k + 2 * m * n)))
+    copies = [(packed.clone(), sw.clone()) for _ in range(n_copies)]
     del packed
     aq = torch.empty((m, k), dtype=torch.uint8, device=dev)
     sa = torch.empty((m,), dtype=torch.float32, device=dev)
-    ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(WEIGHT_COPIES)]
+    ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+          for _ in range(WEIGHT_COPIES if not prefill else 2)]
     ws = S.new_workspace(m, n, k, dev)
 
     def quantize():
         S.sfp8_quantize_rowwise(x_dev, "e4m3", q=aq, scales=sa)
 
     def gemm(j):
-        pk, s = copies[j % WEIGHT_COPIES]
-        S.sfp8_sparse_linear(aq, "e4m3", sa, pk, "e4m3", s, n, k, out=ys[j % WEIGHT_COPIES],
+        pk, s = copies[j % len(copies)]
+        S.sfp8_sparse_linear(aq, "e4m3", sa, pk, "e4m3", s, n, k, out=ys[j % len(ys)],
                              workspace=ws)
 
     def step(j):
@@ -362,7 +381,11 @@ def run_ours(args):
     ms = dist_max(ms, world, dev)
     clocks = clk.summary()
     wbytes = compressed_weight_bytes(n, k)
-    value = world * wbytes * steps / (ms * 1e-3) / 1e9
+    flops = 2.0 * m * n * k
+    if prefill:
+        value = world * flops * steps / (ms * 1e-3) / 1e12
+    else:
+        value = world * wbytes * steps / (ms * 1e-3) / 1e9
 
     # ---- the dominant kernel alone (sparse GEMM), same rotation
     quantize()
@@ -377,6 +400,9 @@ def run_ours(args):
     peak, peak_kind = measured_peaks()
     alg = gemm_algorithmic_bytes(m, n, k)
     achieved = alg / (gemm_us * 1e-6) / 1e9
+    if prefill:
+        peak, peak_kind = measured_tensor_peak()
+        achieved = flops / (gemm_us * 1e-6) / 1e12
     traffic = None
     if NCU_TRAFFIC["sha1"] == kernel_source_sha1():
         traffic = NCU_TRAFFIC["bytes_per_launch"]
@@ -399,14 +425,16 @@ def run_ours(args):
     e1.synchronize()
     ms_e2e = dist_max(e0.elapsed_time(e1), world, dev)
     barrier(world)
-    e2e = {"value": world * wbytes * steps / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+    e2e_value = (world * flops * steps / (ms_e2e * 1e-3) / 1e12 if prefill
+                 else world * wbytes * steps / (ms_e2e * 1e-3) / 1e9)
+    e2e = {"value": e2e_value, "unit": "TFLOP/s" if prefill else "GB/s",
            "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2,
            "ms_per_step": ms_e2e / steps,
            "path": "SparseFp8Linear.forward_host (eager calls, pinned host buffers)"}
 
     # ---- the other decode batch sizes (context lines, same method)
     per_m = {}
-    if args.all_m and world == 1:
+    if args.all_m and world == 1 and not prefill:
         for m2 in (1, 4, 16):
             if m2 == m:
                 continue
@@ -429,21 +457,28 @@ def run_ours(args):
             per_m[str(m2)] = {"value": wbytes * steps / (ms2 * 1e-3) / 1e9, "unit": "GB/s",
                               "ms_per_step": ms2 / steps}
 
+    unit = "TFLOP/s" if prefill else "GB/s"
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "m": m, "k": k, "n": n, "a_dtype": "e4m3",
-                   "w_dtype": "e4m3", "bias": False, "l2": L2_NOTE,
+        "config": {"workload": args.workload, "m": m, "k": k, "n": n, "a_dtype": "e4m3",
+                   "w_dtype": "e4m3", "bias": False,
+                   "l2": L2_NOTE if not prefill else
+                   "rotating %d weight copies; every step's weight is evicted from L2 by the "
+                   "others (%d x %.1f MB + activations and outputs > 126 MB)"
+                   % (len(copies), len(copies), wbytes / 1e6),
                    "step": "sfp8_quantize_rowwise + sfp8_sparse_linear",
                    "weight_bytes_per_step": wbytes, "seeds": seeds,
                    "parallelism": "replica" if world > 1 else "single"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        "roofline": {"bound": "tensor" if prefill else "hbm", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s" if prefill else "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "sparse_linear_kernel<16>" if m <= 16 else "sparse_linear_kernel",
-                     "algorithmic_bytes_per_launch": alg, "us_per_launch": gemm_us,
-                     "peak_source": peak_kind + " hbm_gbs (MEASURED_PEAKS.json)"},
+                     "kernel": "sparse_linear_kernel",
+                     "algorithmic_bytes_per_launch": alg,
+                     "algorithmic_flop_per_launch": flops, "us_per_launch": gemm_us,
+                     "peak_source": peak_kind},
         "quantize_us_per_launch": ms_q * 1e3 / steps,
         "e2e": e2e,
         "gpu_launches": 2 * steps,
@@ -452,7 +487,7 @@ def run_ours(args):
     }
     if per_m:
         line["per_m"] = per_m
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not prefill:
         rate, cores, note, _ = oracle_step_rate(m, seconds=args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": cores, "kind": "oracle",
                                 "sample": note}
@@ -471,6 +506,10 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_8b"],
+                    help="decode gate/up (default, GB/s) or the prefill linears (TFLOP/s)")
+    ap.add_argument("--shape", type=int, default=2, choices=[0, 1, 2, 3],
+                    help="prefill_8b shape: 0 QKV, 1 O, 2 up (default), 3 down")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--all-m", action="store_true", help="also time M=1 and M=4")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -15,8 +15,10 @@ namespace sfp8 {
 // host reads it with sfp8_read_device_status().
 __device__ unsigned int g_device_status;
 
-// Time limit of every pipeline wait, in nanoseconds of %globaltimer.
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// Limit of every pipeline wait, in SM clock cycles (2^31: 1.1 s at 1.965 GHz,
+// 1.6 s at 1.3 GHz).  The SM cycle counter is read because it is cheap; the
+// global timer is a slow read that would delay every stage hand-off.
+constexpr long long kWaitLimitCycles = 1ll << 31;
 
 __device__ __forceinline__ void report_device_error(unsigned int bits) {
   atomicOr(&g_device_status, bits);
@@ -68,17 +70,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase of parity `parity` of barrier `bar` has completed.
-// Gives up after kWaitLimitNs, or as soon as *abort is set by another warp:
-// on a timeout it records SFP8_DEVICE_TIMEOUT and raises *abort.  Returns
-// false when it gave up.
+// Gives up after kWaitLimitCycles, or as soon as *abort is set by another
+// warp: on a timeout it records SFP8_DEVICE_TIMEOUT and raises *abort.
+// Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       report_device_error(SFP8_DEVICE_TIMEOUT);
       *abort = 1;
       return false;
@@ -118,6 +120,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* desc, int 
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
       "l"(desc), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// 3-D tiled TMA load; x innermost (bytes), completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* desc, int x, int y, int z,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(desc), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
       : "memory");
 }
 

@@ -24,7 +24,7 @@ struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
   int num_sms = 0;
-  bool smem_attr_set[16] = {};
+  bool smem_attr_set[32] = {};
 };
 
 std::mutex g_mutex;
@@ -164,9 +164,18 @@ sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64
 
 // ------------------------------------------------------------------ linear plan
 
+constexpr int kSmemLimit = 232448;                 // 227 KB: largest dynamic smem per CTA
+constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice limit
+
 struct LinearPlan {
   int bn;
   int ks;               // k steps per pipeline stage
+  int ra;               // 1: activation resident in shared memory (one token tile)
+  int stages;
+  int producers;
+  int stage_bytes;
+  int ra_bytes;
+  int smem_bytes;
   int whole_tiles;      // 1: each CTA takes whole tiles; 0: stream-K
   int grid;
   int m_tiles;
@@ -207,6 +216,18 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
     const long long waves = (pl.tiles + num_sms - 1) / num_sms;
     pl.whole_tiles = (pl.tiles >= num_sms && pl.tiles * 10 >= 9 * waves * num_sms) ? 1 : 0;
   }
+  // One token tile: keep the CTA's whole activation slice in shared memory
+  // (one copy) when it is small; every stage is then one weight copy.
+  const long long a_slice = static_cast<long long>(pl.bn) * k;
+  pl.ra = (pl.m_tiles == 1 && pl.bn <= 32 && a_slice <= kResidentActMax &&
+           pl.k_steps <= 256) ? 1 : 0;
+  pl.ra_bytes = pl.ra ? static_cast<int>(a_slice) : 0;
+  pl.stage_bytes = pl.ks * kWTileBytes + (pl.ra ? 0 : pl.ks * pl.bn * kStepK);
+  const int budget = kSmemBudget - pl.ra_bytes;
+  pl.stages = budget / pl.stage_bytes;
+  if (pl.stages > 16) pl.stages = 16;
+  pl.producers = kProducerWarps;
+  pl.smem_bytes = linear_smem_bytes(pl.ra_bytes, pl.stages, pl.stage_bytes);
   if (pl.whole_tiles) {
     pl.grid = static_cast<int>(pl.tiles < num_sms ? pl.tiles : num_sms);
     pl.partial_bytes = 0;
@@ -221,39 +242,43 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   return pl;
 }
 
-template <int BN, int KS>
+template <int BN, int KS, bool RA>
 sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const LinearParams& prm,
-                              cudaStream_t st) {
-  using Cfg = LinearCfg<BN, KS>;
-  auto kern = sparse_linear_kernel<BN, KS>;
-  const int slot = (BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 2 + (KS - 1);
+                              int smem_bytes, cudaStream_t st) {
+  auto kern = sparse_linear_kernel<BN, KS, RA>;
+  const int slot =
+      ((BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 2 + (KS - 1)) * 2 +
+      (RA ? 1 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev->smem_attr_set[slot]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Cfg::kSmemBytes) != cudaSuccess)
+                               kSmemLimit) != cudaSuccess)
         return SFP8_ERR_CUDA;
       dev->smem_attr_set[slot] = true;
     }
   }
-  return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), Cfg::kSmemBytes, st, ta, prm);
+  return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), smem_bytes, st, ta, prm);
 }
 
-sfp8_status encode_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                         uint64_t row_stride, uint32_t box_inner, uint32_t box_outer,
-                         CUtensorMapSwizzle swz) {
+// Activation map: dims (128 bytes of k, rows, k steps) with strides (k, 128),
+// so that one box of (128, rows, steps) lands as [step][row][128 B] -- one
+// 128B-swizzled BN x 128 B tile per k step, as the MMA reads it.
+sfp8_status encode_act_3d(CUtensorMap* map, const void* base, uint64_t m, uint64_t k,
+                          uint32_t box_rows, uint32_t box_steps) {
   EncodeTiledFn enc = nullptr;
   sfp8_status s = get_encoder(&enc);
   if (s != SFP8_OK) return s;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_stride};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kStepK), m, k / kStepK};
+  cuuint64_t strides[2] = {k, static_cast<cuuint64_t>(kStepK)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kStepK), box_rows, box_steps};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
 }
+
 
 // Validation shared by the sparse-linear entry points (everything except the
 // workspace); on success fills *plan for the current device.
@@ -289,9 +314,9 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
                           const void* bias, void* y, float* partials, unsigned int* counters,
                           cudaStream_t st) {
   CUtensorMap ta;
-  sfp8_status s = encode_2d_u8(&ta, a_q, static_cast<uint64_t>(k), static_cast<uint64_t>(m),
-                               static_cast<uint64_t>(k), kStepK, static_cast<uint32_t>(pl.bn),
-                               CU_TENSOR_MAP_SWIZZLE_128B);
+  sfp8_status s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
+                                static_cast<uint32_t>(pl.bn),
+                                static_cast<uint32_t>(pl.ra ? pl.k_steps : pl.ks));
   if (s != SFP8_OK) return s;
   LinearParams prm{};
   prm.packed = static_cast<const uint8_t*>(packed);
@@ -311,22 +336,33 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
   prm.iters = pl.iters;
   prm.grid = pl.grid;
   prm.whole_tiles = pl.whole_tiles;
+  prm.stages = pl.stages;
+  prm.ra_bytes = pl.ra_bytes;
+  prm.producers = pl.producers;
   // MMA A operand = weight, B operand = activation.
   prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
                                 kTileN, static_cast<uint32_t>(pl.bn), true);
+  const int sm = pl.smem_bytes;
+  if (pl.ra) {
+    if (pl.ks == 2)
+      return pl.bn == 16 ? launch_linear_cfg<16, 2, true>(dev, ta, prm, sm, st)
+                         : launch_linear_cfg<32, 2, true>(dev, ta, prm, sm, st);
+    return pl.bn == 16 ? launch_linear_cfg<16, 1, true>(dev, ta, prm, sm, st)
+                       : launch_linear_cfg<32, 1, true>(dev, ta, prm, sm, st);
+  }
   if (pl.ks == 2) {
     switch (pl.bn) {
-      case 16: return launch_linear_cfg<16, 2>(dev, ta, prm, st);
-      case 32: return launch_linear_cfg<32, 2>(dev, ta, prm, st);
-      default: return launch_linear_cfg<64, 2>(dev, ta, prm, st);
+      case 16: return launch_linear_cfg<16, 2, false>(dev, ta, prm, sm, st);
+      case 32: return launch_linear_cfg<32, 2, false>(dev, ta, prm, sm, st);
+      default: return launch_linear_cfg<64, 2, false>(dev, ta, prm, sm, st);
     }
   }
   switch (pl.bn) {
-    case 16: return launch_linear_cfg<16, 1>(dev, ta, prm, st);
-    case 32: return launch_linear_cfg<32, 1>(dev, ta, prm, st);
-    case 64: return launch_linear_cfg<64, 1>(dev, ta, prm, st);
-    case 128: return launch_linear_cfg<128, 1>(dev, ta, prm, st);
-    default: return launch_linear_cfg<256, 1>(dev, ta, prm, st);
+    case 16: return launch_linear_cfg<16, 1, false>(dev, ta, prm, sm, st);
+    case 32: return launch_linear_cfg<32, 1, false>(dev, ta, prm, sm, st);
+    case 64: return launch_linear_cfg<64, 1, false>(dev, ta, prm, sm, st);
+    case 128: return launch_linear_cfg<128, 1, false>(dev, ta, prm, sm, st);
+    default: return launch_linear_cfg<256, 1, false>(dev, ta, prm, sm, st);
   }
 }
 

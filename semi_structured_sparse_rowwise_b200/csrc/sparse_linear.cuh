@@ -15,16 +15,22 @@
 // = token m, so in the epilogue the 32 lanes of a warp hold 32 consecutive
 // n of one token and store a contiguous run of y.
 //
-// Structure (one or two CTAs per SM, persistent):
-//   warp 0      producer: per stage of KS 128-wide k steps, ONE contiguous
+// Structure (one CTA per SM, persistent):
+//   warps 0-1   producers: per stage of KS 128-wide k steps, ONE contiguous
 //               bulk copy of KS packed weight tiles (each 8 KB of kept values,
 //               stored pre-swizzled in the 64B-swizzle form the MMA reads,
-//               followed by its 2 KB of index metadata), and KS TMA copies of
-//               the activation tile (BN x 128 B, 128B swizzle).
-//   warp 1      MMA issuer: per k step, copies the metadata block into tensor
+//               followed by its 2 KB of index metadata), and one 3-D TMA copy
+//               of the KS activation tiles (BN x 128 B each, 128B swizzle).
+//               Two producer warps issue, each owning every other stage: a
+//               single issuing thread gets one copy done every ~0.25 us, so
+//               copies from different warps must overlap.
+//               With a single token tile (decode) the CTA's whole activation
+//               slice is loaded once instead (one 3-D TMA copy) and a stage is
+//               just the weight copy.
+//   warp 2      MMA issuer: per k step, copies the metadata block into tensor
 //               memory (tcgen05.cp 128x128b) and issues two 128 x BN x 64
 //               sparse MMAs; frees the stage with tcgen05.commit.
-//   warps 2-5   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
+//   warps 3-6   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
 //               global, or split-K partials to the workspace.
 // Work split, chosen by the host:
 //   whole tiles  CTA c takes tiles c, c + grid, ...: no partial sums.
@@ -53,7 +59,10 @@ constexpr int kStepK = 128;     // logical k per k step
 constexpr int kWValBytes = kTileN * kStepK / 2;       // 8192: kept values of a tile
 constexpr int kWMetaBytes = kTileN * kStepK / 8;      // 2048: index metadata of a tile
 constexpr int kWTileBytes = kWValBytes + kWMetaBytes;  // 10240: packed tile
-constexpr int kGemmThreads = 192;
+constexpr int kProducerWarps = 2;                       // warps issuing copies
+constexpr int kMmaWarp = kProducerWarps;                // one warp issuing MMAs
+constexpr int kEpiWarp0 = kProducerWarps + 1;           // four epilogue warps
+constexpr int kGemmThreads = 32 * (kProducerWarps + 5);
 constexpr int kEpiThreads = 128;
 constexpr int kSmemBudget = 225 * 1024;
 
@@ -63,29 +72,26 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
   return p;
 }
 
-template <int BN, int KS>
+template <int BN, int KS, bool RA>
 struct LinearCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be 16..256, multiple of 16");
   static_assert(KS == 1 || KS == 2, "1 or 2 k steps per stage");
   static constexpr int kATileBytes = BN * kStepK;                 // one k step of activation
-  static constexpr int kStageBytes = KS * (kWTileBytes + kATileBytes);
+  // RA: the activation is resident for the whole k range, not per stage
+  static constexpr int kStageBytes = KS * kWTileBytes + (RA ? 0 : KS * kATileBytes);
   static constexpr int kNumAcc = (2 * BN + 4 * KS <= 512) ? 2 : 1;
   static constexpr int kMetaCol = kNumAcc * BN;
   static constexpr int kTmemCols = pow2_at_least(kNumAcc * BN + 4 * KS);
+  static constexpr int kMaxStages = 16;
   static constexpr int kBarrierBytes = 1024;
-  static constexpr int kStagesMax = 16;
-  // Decode-sized tiles (BN <= 32) use at most half of the SM's shared memory,
-  // so that the next call's CTA can start on the same SM (and stream its
-  // weight) while this one finishes.
-  static constexpr int kBudget = BN <= 32 ? kSmemBudget / 2 - 10 * 1024 : kSmemBudget;
-  static constexpr int kStages =
-      ((kBudget - kBarrierBytes - 1024) / kStageBytes) < kStagesMax
-          ? ((kBudget - kBarrierBytes - 1024) / kStageBytes)
-          : kStagesMax;
-  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kBarrierBytes;
   static_assert(kStageBytes % 1024 == 0, "stages must stay 1024-byte aligned");
-  static_assert(kStages >= 2, "need at least two stages");
 };
+
+// Shared memory of a launch: align slack + resident activation + stages +
+// barriers.
+__host__ __device__ constexpr int linear_smem_bytes(int ra_bytes, int stages, int stage_bytes) {
+  return 1024 + ra_bytes + stages * stage_bytes + 1024;
+}
 
 struct LinearParams {
   const uint8_t* packed;    // compressed weight, 10 KB tiles (layout version 3)
@@ -103,6 +109,9 @@ struct LinearParams {
   long long iters;          // tiles * units
   int grid;
   int whole_tiles;          // 1: CTA c takes tiles c, c + grid, ...; 0: stream-K
+  int stages;               // shared-memory pipeline depth (<= kMaxStages)
+  int ra_bytes;             // resident activation bytes (BN * k) or 0
+  int producers;            // producer warps issuing copies (1..kProducerWarps)
   uint32_t idesc;
 };
 
@@ -178,23 +187,26 @@ __device__ __forceinline__ void load_sa(const LinearParams& p, int m0, float (&s
   for (int j = 0; j < 16; ++j) sa[j] = (m0 + j < p.m) ? __ldg(p.s_a + m0 + j) : 0.0f;
 }
 
-template <int BN, int KS>
+template <int BN, int KS, bool RA>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_a, const LinearParams p) {
-  using Cfg = LinearCfg<BN, KS>;
-  constexpr int S = Cfg::kStages;
+  using Cfg = LinearCfg<BN, KS, RA>;
+  const int S = p.stages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cfg::kStageBytes);
+  uint8_t* ra_base = smem;                       // resident activation (RA)
+  uint8_t* stage_base = smem + p.ra_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage_base + S * Cfg::kStageBytes);
+  constexpr int SM = Cfg::kMaxStages;
   uint64_t* full_bar = bars;                  // [S]
-  uint64_t* empty_bar = bars + S;             // [S]
-  uint64_t* accf_bar = bars + 2 * S;          // [2]
-  uint64_t* acce_bar = bars + 2 * S + 2;      // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 5);
-  uint64_t* drain_bar = bars + 2 * S + 6;
+  uint64_t* empty_bar = bars + SM;            // [S]
+  uint64_t* accf_bar = bars + 2 * SM;         // [2]
+  uint64_t* acce_bar = bars + 2 * SM + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SM + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * SM + 5);
+  uint64_t* drain_bar = bars + 2 * SM + 6;
+  uint64_t* ra_bar = bars + 2 * SM + 7;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -215,11 +227,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(smem_u32(&acce_bar[b]), kEpiThreads / 32);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    mbar_init(smem_u32(ra_bar), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_a);
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     tmem_relinquish();
   }
@@ -228,9 +241,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < kProducerWarps) {
+    // ------------------------------------------------------------ producers
+    // Lane 0 of producer warp w < P issues the copies of stages i with
+    // i % P == w.
+    const int P = p.producers;
+    const int pw = warp;
+    if (lane == 0 && pw < P) {
       // A weight tile is read once when there is one token tile (decode:
       // keep it from displacing anything); otherwise every token tile reuses
       // it, so it must stay in L2.
@@ -248,11 +265,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       auto issue_act = [&](int stage, long long tile, int u) {
         const int mt = static_cast<int>(tile % p.m_tiles);
         uint8_t* st = stage_base + stage * Cfg::kStageBytes + KS * kWTileBytes;
-        const uint32_t fb = smem_u32(&full_bar[stage]);
-#pragma unroll
-        for (int j = 0; j < KS; ++j)
-          tma_load_2d(smem_u32(st + j * Cfg::kATileBytes), &tm_a, (u * KS + j) * kStepK,
-                      mt * BN, fb, pol_a);
+        tma_load_3d(smem_u32(st), &tm_a, 0, mt * BN, u * KS, smem_u32(&full_bar[stage]), pol_a);
       };
       // The weight does not depend on the preceding kernel: fill the first
       // stages with weight tiles before waiting for the activation.
@@ -263,48 +276,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int a0, a1;
         while (pre_count < S && pre.next(t2, a0, a1))
           for (int u = a0; u < a1 && pre_count < S; ++u) {
-            issue_weight(static_cast<int>(pre_count), t2, u);
+            if (pre_count % P == pw) issue_weight(static_cast<int>(pre_count), t2, u);
             ++pre_count;
           }
       }
       grid_dependency_wait();
+      if (RA && pw == 0) {
+        // the whole activation slice of this CTA: [k steps][BN rows][128 B]
+        mbar_arrive_expect_tx(smem_u32(ra_bar), p.ra_bytes);
+        tma_load_3d(smem_u32(ra_base), &tm_a, 0, 0, 0, smem_u32(ra_bar), pol_a);
+      }
       SegmentWalker walk(p, cta);
       long long tile;
       int u0, u1;
-      int stage = 0;
-      uint32_t phase = 0;
-      long long issued = 0;
+      long long i = 0;              // stage sequence number
       bool ok = true;
       while (ok && walk.next(tile, u0, u1)) {
-        for (int u = u0; u < u1; ++u) {
-          if (issued >= pre_count) {
+        for (int u = u0; u < u1; ++u, ++i) {
+          if (i % P != pw) continue;
+          const int stage = static_cast<int>(i % S);
+          if (i >= pre_count) {
+            const uint32_t phase = static_cast<uint32_t>((i / S) & 1);
             if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag)) {
               ok = false;
               break;
             }
             issue_weight(stage, tile, u);
           }
-          issue_act(stage, tile, u);
-          ++issued;
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          if (!RA) issue_act(stage, tile, u);
         }
       }
       if (!ok) {
-        // Let the copies already issued land before the CTA exits.  Stage s
-        // was last filled by one of the last min(S, issued) iterations.
+        // Let this lane's copies already issued land before the CTA exits.
+        const long long issued = i;      // stages up to (not incl.) i were considered
         long long first = issued > S ? issued - S : 0;
-        for (long long i = first; i < issued; ++i) {
-          const int s = static_cast<int>(i % S);
-          const uint32_t ph = static_cast<uint32_t>((i / S) & 1);
+        for (long long t = first; t < issued; ++t) {
+          if (t % P != pw) continue;
+          const int s2 = static_cast<int>(t % S);
+          const uint32_t ph = static_cast<uint32_t>((t / S) & 1);
           volatile int no_abort = 0;
-          mbar_wait(smem_u32(&full_bar[s]), ph, &no_abort);
+          mbar_wait(smem_u32(&full_bar[s2]), ph, &no_abort);
+        }
+        if (RA && pw == 0) {
+          volatile int no_abort = 0;
+          mbar_wait(smem_u32(ra_bar), 0, &no_abort);
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       grid_dependency_wait();   // start the wait limits only once inputs exist
@@ -317,6 +336,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       const uint32_t e_tmem = tmem_base + Cfg::kMetaCol;
       bool ok = true;
+      if (RA) ok = mbar_wait(smem_u32(ra_bar), 0, abort_flag);
       while (ok && walk.next(tile, u0, u1)) {
         if (!mbar_wait(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
@@ -332,7 +352,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int j = 0; j < KS; ++j) {
             const uint32_t w_addr = st + j * kWTileBytes;
             const uint32_t e_addr = w_addr + kWValBytes;
-            const uint32_t a_addr = st + KS * kWTileBytes + j * Cfg::kATileBytes;
+            const uint32_t a_addr =
+                RA ? smem_u32(ra_base) + (u * KS + j) * Cfg::kATileBytes
+                   : st + KS * kWTileBytes + j * Cfg::kATileBytes;
             // metadata: 128 rows x 16 bytes, no swizzle, 8-row groups 128 B apart
             tc_cp_128x128b(e_tmem + 4 * j, smem_desc(e_addr, 0, 128, kNoSwizzle));
 #pragma unroll
@@ -515,7 +537,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   // ------------------------------------------------------------ teardown
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::kTmemCols);
   }
