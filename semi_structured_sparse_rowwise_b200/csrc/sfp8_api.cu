@@ -24,7 +24,7 @@ struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
   int num_sms = 0;
-  bool smem_attr_set[32] = {};
+  bool smem_attr_set[32] = {};   // (BN, KS, RA) instantiations
 };
 
 std::mutex g_mutex;
@@ -166,6 +166,7 @@ sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64
 
 constexpr int kSmemLimit = 232448;                 // 227 KB: largest dynamic smem per CTA
 constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice limit
+constexpr int kPlanProducers = 4;                  // producer warps used
 
 struct LinearPlan {
   int bn;
@@ -201,8 +202,11 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   pl.bn = choose_bn(m);
   pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
   pl.k_steps = static_cast<int>(k / kStepK);
-  // Two k steps per stage (one 20 KB weight copy) when the stage stays small.
-  pl.ks = (pl.bn <= 64 && pl.k_steps % 2 == 0) ? 2 : 1;
+  // Several k steps per stage (one 20-40 KB weight copy) when the stage stays
+  // small: an issuing thread keeps about one copy in flight, so bytes per
+  // copy set the rate.
+  pl.ks = (pl.bn <= 32 && pl.k_steps % 4 == 0) ? 4
+        : (pl.bn <= 64 && pl.k_steps % 2 == 0) ? 2 : 1;
   pl.units = pl.k_steps / pl.ks;
   pl.n_tiles = (n + kTileN - 1) / kTileN;
   pl.tiles = pl.n_tiles * pl.m_tiles;
@@ -226,7 +230,7 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   const int budget = kSmemBudget - pl.ra_bytes;
   pl.stages = budget / pl.stage_bytes;
   if (pl.stages > 16) pl.stages = 16;
-  pl.producers = kProducerWarps;
+  pl.producers = kPlanProducers;
   pl.smem_bytes = linear_smem_bytes(pl.ra_bytes, pl.stages, pl.stage_bytes);
   if (pl.whole_tiles) {
     pl.grid = static_cast<int>(pl.tiles < num_sms ? pl.tiles : num_sms);
@@ -247,8 +251,8 @@ sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const Line
                               int smem_bytes, cudaStream_t st) {
   auto kern = sparse_linear_kernel<BN, KS, RA>;
   const int slot =
-      ((BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 2 + (KS - 1)) * 2 +
-      (RA ? 1 : 0);
+      ((BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 3 +
+       (KS == 1 ? 0 : KS == 2 ? 1 : 2)) * 2 + (RA ? 1 : 0);
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!dev->smem_attr_set[slot]) {
@@ -344,24 +348,25 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
                                 kTileN, static_cast<uint32_t>(pl.bn), true);
   const int sm = pl.smem_bytes;
   if (pl.ra) {
-    if (pl.ks == 2)
-      return pl.bn == 16 ? launch_linear_cfg<16, 2, true>(dev, ta, prm, sm, st)
-                         : launch_linear_cfg<32, 2, true>(dev, ta, prm, sm, st);
-    return pl.bn == 16 ? launch_linear_cfg<16, 1, true>(dev, ta, prm, sm, st)
-                       : launch_linear_cfg<32, 1, true>(dev, ta, prm, sm, st);
-  }
-  if (pl.ks == 2) {
-    switch (pl.bn) {
-      case 16: return launch_linear_cfg<16, 2, false>(dev, ta, prm, sm, st);
-      case 32: return launch_linear_cfg<32, 2, false>(dev, ta, prm, sm, st);
-      default: return launch_linear_cfg<64, 2, false>(dev, ta, prm, sm, st);
+    switch (pl.bn * 8 + pl.ks) {
+      case 16 * 8 + 1: return launch_linear_cfg<16, 1, true>(dev, ta, prm, sm, st);
+      case 16 * 8 + 2: return launch_linear_cfg<16, 2, true>(dev, ta, prm, sm, st);
+      case 16 * 8 + 4: return launch_linear_cfg<16, 4, true>(dev, ta, prm, sm, st);
+      case 32 * 8 + 1: return launch_linear_cfg<32, 1, true>(dev, ta, prm, sm, st);
+      case 32 * 8 + 2: return launch_linear_cfg<32, 2, true>(dev, ta, prm, sm, st);
+      default: return launch_linear_cfg<32, 4, true>(dev, ta, prm, sm, st);
     }
   }
-  switch (pl.bn) {
-    case 16: return launch_linear_cfg<16, 1, false>(dev, ta, prm, sm, st);
-    case 32: return launch_linear_cfg<32, 1, false>(dev, ta, prm, sm, st);
-    case 64: return launch_linear_cfg<64, 1, false>(dev, ta, prm, sm, st);
-    case 128: return launch_linear_cfg<128, 1, false>(dev, ta, prm, sm, st);
+  switch (pl.bn * 8 + pl.ks) {
+    case 16 * 8 + 1: return launch_linear_cfg<16, 1, false>(dev, ta, prm, sm, st);
+    case 16 * 8 + 2: return launch_linear_cfg<16, 2, false>(dev, ta, prm, sm, st);
+    case 16 * 8 + 4: return launch_linear_cfg<16, 4, false>(dev, ta, prm, sm, st);
+    case 32 * 8 + 1: return launch_linear_cfg<32, 1, false>(dev, ta, prm, sm, st);
+    case 32 * 8 + 2: return launch_linear_cfg<32, 2, false>(dev, ta, prm, sm, st);
+    case 32 * 8 + 4: return launch_linear_cfg<32, 4, false>(dev, ta, prm, sm, st);
+    case 64 * 8 + 1: return launch_linear_cfg<64, 1, false>(dev, ta, prm, sm, st);
+    case 64 * 8 + 2: return launch_linear_cfg<64, 2, false>(dev, ta, prm, sm, st);
+    case 128 * 8 + 1: return launch_linear_cfg<128, 1, false>(dev, ta, prm, sm, st);
     default: return launch_linear_cfg<256, 1, false>(dev, ta, prm, sm, st);
   }
 }

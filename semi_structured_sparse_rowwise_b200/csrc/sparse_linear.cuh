@@ -16,21 +16,21 @@
 // n of one token and store a contiguous run of y.
 //
 // Structure (one CTA per SM, persistent):
-//   warps 0-1   producers: per stage of KS 128-wide k steps, ONE contiguous
+//   warps 0-3   producers: per stage of KS 128-wide k steps, ONE contiguous
 //               bulk copy of KS packed weight tiles (each 8 KB of kept values,
 //               stored pre-swizzled in the 64B-swizzle form the MMA reads,
 //               followed by its 2 KB of index metadata), and one 3-D TMA copy
 //               of the KS activation tiles (BN x 128 B each, 128B swizzle).
-//               Two producer warps issue, each owning every other stage: a
-//               single issuing thread gets one copy done every ~0.25 us, so
-//               copies from different warps must overlap.
+//               Up to four producer warps issue, each owning every P-th
+//               stage: an issuing thread keeps about one copy in flight, so
+//               copies must come from several warps to overlap.
 //               With a single token tile (decode) the CTA's whole activation
 //               slice is loaded once instead (one 3-D TMA copy) and a stage is
 //               just the weight copy.
-//   warp 2      MMA issuer: per k step, copies the metadata block into tensor
+//   warp 4      MMA issuer: per k step, copies the metadata block into tensor
 //               memory (tcgen05.cp 128x128b) and issues two 128 x BN x 64
 //               sparse MMAs; frees the stage with tcgen05.commit.
-//   warps 3-6   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
+//   warps 5-8   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
 //               global, or split-K partials to the workspace.
 // Work split, chosen by the host:
 //   whole tiles  CTA c takes tiles c, c + grid, ...: no partial sums.
@@ -59,7 +59,7 @@ constexpr int kStepK = 128;     // logical k per k step
 constexpr int kWValBytes = kTileN * kStepK / 2;       // 8192: kept values of a tile
 constexpr int kWMetaBytes = kTileN * kStepK / 8;      // 2048: index metadata of a tile
 constexpr int kWTileBytes = kWValBytes + kWMetaBytes;  // 10240: packed tile
-constexpr int kProducerWarps = 2;                       // warps issuing copies
+constexpr int kProducerWarps = 4;                       // warps issuing copies (max)
 constexpr int kMmaWarp = kProducerWarps;                // one warp issuing MMAs
 constexpr int kEpiWarp0 = kProducerWarps + 1;           // four epilogue warps
 constexpr int kGemmThreads = 32 * (kProducerWarps + 5);
@@ -75,7 +75,7 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
 template <int BN, int KS, bool RA>
 struct LinearCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN must be 16..256, multiple of 16");
-  static_assert(KS == 1 || KS == 2, "1 or 2 k steps per stage");
+  static_assert(KS == 1 || KS == 2 || KS == 4, "1, 2 or 4 k steps per stage");
   static constexpr int kATileBytes = BN * kStepK;                 // one k step of activation
   // RA: the activation is resident for the whole k range, not per stage
   static constexpr int kStageBytes = KS * kWTileBytes + (RA ? 0 : KS * kATileBytes);
@@ -280,11 +280,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ++pre_count;
           }
       }
-      grid_dependency_wait();
-      if (RA && pw == 0) {
-        // the whole activation slice of this CTA: [k steps][BN rows][128 B]
+      if (RA && pw == P - 1) {
+        // The whole activation slice of this CTA, [k steps][BN rows][128 B],
+        // in one copy by the warp that issued the fewest prefetch copies.
+        grid_dependency_wait();
         mbar_arrive_expect_tx(smem_u32(ra_bar), p.ra_bytes);
         tma_load_3d(smem_u32(ra_base), &tm_a, 0, 0, 0, smem_u32(ra_bar), pol_a);
+      } else {
+        grid_dependency_wait();
       }
       SegmentWalker walk(p, cta);
       long long tile;
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           volatile int no_abort = 0;
           mbar_wait(smem_u32(&full_bar[s2]), ph, &no_abort);
         }
-        if (RA && pw == 0) {
+        if (RA && pw == P - 1) {
           volatile int no_abort = 0;
           mbar_wait(smem_u32(ra_bar), 0, &no_abort);
         }
