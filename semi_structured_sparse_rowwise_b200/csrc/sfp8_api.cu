@@ -14,6 +14,7 @@
 #include "quantize_rowwise.cuh"
 #include "sparse24_pack.cuh"
 #include "sparse_linear.cuh"
+#include "sparse_linear_pair.cuh"
 
 namespace sfp8 {
 namespace {
@@ -25,6 +26,7 @@ struct DeviceInfo {
   bool is_sm100 = false;
   int num_sms = 0;
   bool smem_attr_set[32] = {};   // (BN, KS, RA) instantiations
+  int pair_clusters[3] = {};     // co-resident CTA pairs of the pair kernel, by KS (0: unknown)
 };
 
 std::mutex g_mutex;
@@ -169,6 +171,7 @@ constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice 
 constexpr int kPlanProducers = 4;                  // producer warps used
 
 struct LinearPlan {
+  int pair;             // 1: the CTA-pair kernel (256 x 256 tiles)
   int bn;
   int ks;               // k steps per pipeline stage
   int ra;               // 1: activation resident in shared memory (one token tile)
@@ -197,8 +200,34 @@ int choose_bn(int64_t m) {
   return 128;
 }
 
+// Token count from which the CTA-pair kernel is used.
+constexpr int64_t kPairMinTokens = 512;
+
 LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   LinearPlan pl{};
+  if (m >= kPairMinTokens) {
+    pl.pair = 1;
+    // Tokens per tile: the fewest tiles of at most kPairMaxTokens, split
+    // evenly (rounded up to the pair MMA's N granularity of 32).
+    const int64_t mt = (m + kPairMaxTokens - 1) / kPairMaxTokens;
+    pl.bn = static_cast<int>(((m + mt - 1) / mt + 31) / 32 * 32);
+    pl.ks = 1;
+    pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
+    pl.k_steps = static_cast<int>(k / kStepK);
+    pl.units = pl.k_steps / pl.ks;
+    pl.n_tiles = (n + kTileN - 1) / kTileN;
+    pl.tiles = ((pl.n_tiles + 1) / 2) * pl.m_tiles;
+    pl.iters = pl.tiles * pl.units;
+    pl.whole_tiles = 1;
+    pl.stage_bytes = PairCfg<1>::stage_bytes(pl.bn);
+    pl.stages = kSmemBudget / pl.stage_bytes;
+    if (pl.stages > PairCfg<1>::kMaxStages) pl.stages = PairCfg<1>::kMaxStages;
+    pl.producers = kPlanProducers;
+    pl.smem_bytes = pair_smem_bytes(pl.stages, pl.stage_bytes);
+    // The grid (pairs) is set at launch from the co-resident cluster count.
+    pl.grid = 2 * static_cast<int>(pl.tiles < num_sms / 2 ? pl.tiles : num_sms / 2);
+    return pl;
+  }
   pl.bn = choose_bn(m);
   pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
   pl.k_steps = static_cast<int>(k / kStepK);
@@ -265,6 +294,24 @@ sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const Line
   return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), smem_bytes, st, ta, prm);
 }
 
+// Weight map for the pair kernel: the packed buffer as (256 B, 40, tiles x
+// k steps) bytes, so that a box (256, 40, KS) is KS consecutive 10 KB packed
+// tiles, landing in shared memory exactly as stored (no swizzle).
+sfp8_status encode_weight_3d(CUtensorMap* map, const void* packed, uint64_t n_tiles,
+                             uint64_t k_steps, uint32_t box_steps) {
+  EncodeTiledFn enc = nullptr;
+  sfp8_status s = get_encoder(&enc);
+  if (s != SFP8_OK) return s;
+  cuuint64_t dims[3] = {256, kWTileBytes / 256, n_tiles * k_steps};
+  cuuint64_t strides[2] = {256, kWTileBytes};
+  cuuint32_t box[3] = {256, kWTileBytes / 256, box_steps};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
+}
+
 // Activation map: dims (128 bytes of k, rows, k steps) with strides (k, 128),
 // so that one box of (128, rows, steps) lands as [step][row][128 B] -- one
 // 128B-swizzled BN x 128 B tile per k step, as the MMA reads it.
@@ -311,12 +358,80 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
   return SFP8_OK;
 }
 
+// CTA-pair GEMM: both maps, the co-resident pair count (queried once per
+// device), launch with programmatic stream serialisation.
+sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
+                        sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
+                        sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
+                        const void* bias, void* y, cudaStream_t st) {
+  auto kern = sparse_linear_pair_kernel<1>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (dev->pair_clusters[1] == 0) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+          cudaSuccess)
+        return SFP8_ERR_CUDA;
+      cudaLaunchConfig_t qc{};
+      qc.gridDim = dim3(2 * (dev->num_sms / 2));
+      qc.blockDim = dim3(kPairThreads);
+      qc.dynamicSmemBytes = pl.smem_bytes;
+      cudaLaunchAttribute ca[1];
+      ca[0].id = cudaLaunchAttributeClusterDimension;
+      ca[0].val.clusterDim.x = 2;
+      ca[0].val.clusterDim.y = 1;
+      ca[0].val.clusterDim.z = 1;
+      qc.attrs = ca;
+      qc.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &qc) != cudaSuccess || clusters < 1) {
+        cudaGetLastError();
+        return SFP8_ERR_CUDA;
+      }
+      dev->pair_clusters[1] = clusters;
+    }
+  }
+  CUtensorMap tw, ta;
+  sfp8_status s = encode_weight_3d(&tw, packed, static_cast<uint64_t>(pl.n_tiles),
+                                   static_cast<uint64_t>(pl.k_steps), 1);
+  if (s != SFP8_OK) return s;
+  s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
+                    static_cast<uint32_t>(pl.bn / 2), 1);
+  if (s != SFP8_OK) return s;
+  const long long max_pairs = dev->pair_clusters[1];
+  const int pairs = static_cast<int>(pl.tiles < max_pairs ? pl.tiles : max_pairs);
+  PairParams prm{};
+  prm.s_a = s_a;
+  prm.s_w = s_w;
+  prm.bias = static_cast<const __nv_bfloat16*>(bias);
+  prm.y = static_cast<__nv_bfloat16*>(y);
+  prm.m = static_cast<int>(m);
+  prm.n = static_cast<int>(n);
+  prm.k = static_cast<int>(k);
+  prm.n_tiles = static_cast<int>(pl.n_tiles);
+  prm.n_pairs = static_cast<int>((pl.n_tiles + 1) / 2);
+  prm.bn = pl.bn;
+  prm.m_tiles = pl.m_tiles;
+  prm.k_steps = pl.k_steps;
+  prm.units = pl.units;
+  prm.tiles = static_cast<int>(pl.tiles);
+  prm.pairs = pairs;
+  prm.stages = pl.stages;
+  prm.stage_bytes = pl.stage_bytes;
+  prm.producers = pl.producers;
+  prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
+                                kPairTileN, static_cast<uint32_t>(pl.bn), true);
+  return launch_dependent(kern, dim3(2 * pairs), dim3(kPairThreads), pl.smem_bytes, st, tw, ta,
+                          prm);
+}
+
 // Encodes the activation map and launches the GEMM for a validated plan.
 sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
                           sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
                           sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
                           const void* bias, void* y, float* partials, unsigned int* counters,
                           cudaStream_t st) {
+  if (pl.pair)
+    return launch_pair(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y, st);
   CUtensorMap ta;
   sfp8_status s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
                                 static_cast<uint32_t>(pl.bn),

@@ -64,6 +64,39 @@ def test_ragged_multi_tile(m, k, n, pair):
     run_full(x, w, a_fmt, w_fmt, b)
 
 
+# Shapes for the CTA-pair kernel (512 tokens and more): an odd count of
+# 128-row weight tiles (the second CTA of the last pair has no rows), ragged
+# token tiles, a single k step, and token counts that choose different tile
+# widths (192, 224).
+PAIR_SHAPES = [(512, 128, 100), (700, 384, 390), (1000, 256, 1000), (2049, 128, 260),
+               (600, 640, 129)]
+
+
+@pytest.mark.parametrize("m,k,n", PAIR_SHAPES)
+@pytest.mark.parametrize("pair", PAIRS)
+def test_pair_kernel_shapes(m, k, n, pair):
+    a_fmt, w_fmt = pair
+    seed = 9100 + m * 5 + k * 3 + n
+    x = synthetic.activation(seed, m, k, dist="student_t3", zero_row_frac=0.03)
+    w = synthetic.weight(seed + 1, n, k, neg_zero_frac=0.02)
+    b = synthetic.bias(seed + 2, n) if (m + n) % 2 else None
+    run_full(x, w, a_fmt, w_fmt, b)
+
+
+def test_pair_kernel_deterministic():
+    m, k, n = 1000, 512, 700
+    x = synthetic.activation(31, m, k)
+    w = synthetic.weight(32, n, k)
+    gl = GpuLayer(w, "e4m3")
+    aq, sa = S.sfp8_quantize_rowwise(bf16_dev(x), "e4m3")
+    assert S.sfp8_sparse_linear_workspace_bytes(m, n, k) == 0
+    y1 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.packed, "e4m3", gl.sw, n, k)
+    y2 = S.sfp8_sparse_linear(aq, "e4m3", sa, gl.packed, "e4m3", gl.sw, n, k)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    _status_clean()
+
+
 def test_deterministic_and_counters_reset():
     m, k, n = 40, 1024, 700            # split-K tiles (grid > tiles)
     x = synthetic.activation(1, m, k)
