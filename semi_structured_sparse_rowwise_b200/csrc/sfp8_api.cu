@@ -202,6 +202,8 @@ int choose_bn(int64_t m) {
 
 // Token count from which the CTA-pair kernel is used.
 constexpr int64_t kPairMinTokens = 512;
+// k steps per pipeline stage of the CTA-pair kernel (when k allows).
+constexpr int kPairStepsPerStage = 2;
 
 LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   LinearPlan pl{};
@@ -211,15 +213,15 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
     // evenly (rounded up to the pair MMA's N granularity of 32).
     const int64_t mt = (m + kPairMaxTokens - 1) / kPairMaxTokens;
     pl.bn = static_cast<int>(((m + mt - 1) / mt + 31) / 32 * 32);
-    pl.ks = 1;
     pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
     pl.k_steps = static_cast<int>(k / kStepK);
+    pl.ks = (kPairStepsPerStage == 2 && pl.k_steps % 2 == 0) ? 2 : 1;
     pl.units = pl.k_steps / pl.ks;
     pl.n_tiles = (n + kTileN - 1) / kTileN;
     pl.tiles = ((pl.n_tiles + 1) / 2) * pl.m_tiles;
     pl.iters = pl.tiles * pl.units;
     pl.whole_tiles = 1;
-    pl.stage_bytes = PairCfg<1>::stage_bytes(pl.bn);
+    pl.stage_bytes = pl.ks == 2 ? PairCfg<2>::stage_bytes(pl.bn) : PairCfg<1>::stage_bytes(pl.bn);
     pl.stages = kSmemBudget / pl.stage_bytes;
     if (pl.stages > PairCfg<1>::kMaxStages) pl.stages = PairCfg<1>::kMaxStages;
     pl.producers = kPlanProducers;
@@ -231,11 +233,12 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   pl.bn = choose_bn(m);
   pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
   pl.k_steps = static_cast<int>(k / kStepK);
-  // Several k steps per stage (one 20-40 KB weight copy) when the stage stays
-  // small: an issuing thread keeps about one copy in flight, so bytes per
-  // copy set the rate.
+  // Several k steps per stage (20-50 KB): the stages are consumed in order,
+  // and fewer, larger copies keep more bytes in flight per SM than many
+  // small ones (measured on B200: the feed rate per SM grows with the copy
+  // size at a fixed shared-memory ring).
   pl.ks = (pl.bn <= 32 && pl.k_steps % 4 == 0) ? 4
-        : (pl.bn <= 64 && pl.k_steps % 2 == 0) ? 2 : 1;
+        : (pl.bn <= 128 && pl.k_steps % 2 == 0) ? 2 : 1;
   pl.units = pl.k_steps / pl.ks;
   pl.n_tiles = (n + kTileN - 1) / kTileN;
   pl.tiles = pl.n_tiles * pl.m_tiles;
@@ -360,21 +363,22 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
 
 // CTA-pair GEMM: both maps, the co-resident pair count (queried once per
 // device), launch with programmatic stream serialisation.
-sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
-                        sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
-                        sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
-                        const void* bias, void* y, cudaStream_t st) {
-  auto kern = sparse_linear_pair_kernel<1>;
+template <int KS>
+sfp8_status launch_pair_ks(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
+                           sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
+                           sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
+                           const void* bias, void* y, cudaStream_t st) {
+  auto kern = sparse_linear_pair_kernel<KS>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (dev->pair_clusters[1] == 0) {
+    if (dev->pair_clusters[KS] == 0) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
           cudaSuccess)
         return SFP8_ERR_CUDA;
       cudaLaunchConfig_t qc{};
       qc.gridDim = dim3(2 * (dev->num_sms / 2));
       qc.blockDim = dim3(kPairThreads);
-      qc.dynamicSmemBytes = pl.smem_bytes;
+      qc.dynamicSmemBytes = kSmemLimit;
       cudaLaunchAttribute ca[1];
       ca[0].id = cudaLaunchAttributeClusterDimension;
       ca[0].val.clusterDim.x = 2;
@@ -387,17 +391,17 @@ sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
         cudaGetLastError();
         return SFP8_ERR_CUDA;
       }
-      dev->pair_clusters[1] = clusters;
+      dev->pair_clusters[KS] = clusters;
     }
   }
   CUtensorMap tw, ta;
   sfp8_status s = encode_weight_3d(&tw, packed, static_cast<uint64_t>(pl.n_tiles),
-                                   static_cast<uint64_t>(pl.k_steps), 1);
+                                   static_cast<uint64_t>(pl.k_steps), KS);
   if (s != SFP8_OK) return s;
   s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
-                    static_cast<uint32_t>(pl.bn / 2), 1);
+                    static_cast<uint32_t>(pl.bn / 2), KS);
   if (s != SFP8_OK) return s;
-  const long long max_pairs = dev->pair_clusters[1];
+  const long long max_pairs = dev->pair_clusters[KS];
   const int pairs = static_cast<int>(pl.tiles < max_pairs ? pl.tiles : max_pairs);
   PairParams prm{};
   prm.s_a = s_a;
@@ -422,6 +426,17 @@ sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
                                 kPairTileN, static_cast<uint32_t>(pl.bn), true);
   return launch_dependent(kern, dim3(2 * pairs), dim3(kPairThreads), pl.smem_bytes, st, tw, ta,
                           prm);
+}
+
+sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
+                        sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
+                        sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
+                        const void* bias, void* y, cudaStream_t st) {
+  if (pl.ks == 2)
+    return launch_pair_ks<2>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                             st);
+  return launch_pair_ks<1>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                           st);
 }
 
 // Encodes the activation map and launches the GEMM for a validated plan.
@@ -469,7 +484,8 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
       case 16 * 8 + 4: return launch_linear_cfg<16, 4, true>(dev, ta, prm, sm, st);
       case 32 * 8 + 1: return launch_linear_cfg<32, 1, true>(dev, ta, prm, sm, st);
       case 32 * 8 + 2: return launch_linear_cfg<32, 2, true>(dev, ta, prm, sm, st);
-      default: return launch_linear_cfg<32, 4, true>(dev, ta, prm, sm, st);
+      case 32 * 8 + 4: return launch_linear_cfg<32, 4, true>(dev, ta, prm, sm, st);
+      default: return SFP8_ERR_UNSUPPORTED_SHAPE;   // no such plan is made
     }
   }
   switch (pl.bn * 8 + pl.ks) {
@@ -482,7 +498,8 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
     case 64 * 8 + 1: return launch_linear_cfg<64, 1, false>(dev, ta, prm, sm, st);
     case 64 * 8 + 2: return launch_linear_cfg<64, 2, false>(dev, ta, prm, sm, st);
     case 128 * 8 + 1: return launch_linear_cfg<128, 1, false>(dev, ta, prm, sm, st);
-    default: return launch_linear_cfg<256, 1, false>(dev, ta, prm, sm, st);
+    case 128 * 8 + 2: return launch_linear_cfg<128, 2, false>(dev, ta, prm, sm, st);
+    default: return SFP8_ERR_UNSUPPORTED_SHAPE;   // no such plan is made
   }
 }
 
