@@ -365,6 +365,17 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void* desc,
       : "memory");
 }
 
+// 4-D form of tma_load_3d_pair.
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* desc, int x, int y,
+                                                 int z, int w, uint32_t bar_cluster,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx"
+      "::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(desc), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar_cluster), "l"(policy)
+      : "memory");
+}
+
 // Tensor memory of a CTA pair: one warp with the same warp index in each CTA
 // issues these, with the same shared-memory slot.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {

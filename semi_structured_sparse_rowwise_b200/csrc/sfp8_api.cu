@@ -26,7 +26,7 @@ struct DeviceInfo {
   bool is_sm100 = false;
   int num_sms = 0;
   bool smem_attr_set[32] = {};   // (BN, KS, RA) instantiations
-  int pair_clusters[3] = {};     // co-resident CTA pairs of the pair kernel, by KS (0: unknown)
+  int pair_clusters[4] = {};     // co-resident pairs of the pair kernel by (KS, WT) (0: unknown)
 };
 
 std::mutex g_mutex;
@@ -171,7 +171,8 @@ constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice 
 constexpr int kPlanProducers = 4;                  // producer warps used
 
 struct LinearPlan {
-  int pair;             // 1: the CTA-pair kernel (256 x 256 tiles)
+  int pair;             // 1: the CTA-pair kernel
+  int wt;               // pair kernel: weight tiles (128 rows) per CTA
   int bn;
   int ks;               // k steps per pipeline stage
   int ra;               // 1: activation resident in shared memory (one token tile)
@@ -200,10 +201,20 @@ int choose_bn(int64_t m) {
   return 128;
 }
 
+// Producer warps for a ring of `stages` stages.  Producer w issues stages
+// i = w (mod P) into ring slot i mod stages and waits on the slot's
+// phase parity; with no more producers than slots, a producer is never two
+// phases ahead of a slot, so the parity it waits on is unambiguous.
+int producers_for(int stages) { return stages < kPlanProducers ? stages : kPlanProducers; }
+
 // Token count from which the CTA-pair kernel is used.
 constexpr int64_t kPairMinTokens = 512;
 // k steps per pipeline stage of the CTA-pair kernel (when k allows).
 constexpr int kPairStepsPerStage = 2;
+// Weight tiles per CTA of the CTA-pair kernel (when there are enough tiles
+// and k is long enough).
+constexpr int kPairWeightTiles = 2;
+constexpr int kPairTwoTileMinSteps = 64;   // k >= 8192
 
 LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   LinearPlan pl{};
@@ -218,13 +229,20 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
     pl.ks = (kPairStepsPerStage == 2 && pl.k_steps % 2 == 0) ? 2 : 1;
     pl.units = pl.k_steps / pl.ks;
     pl.n_tiles = (n + kTileN - 1) / kTileN;
-    pl.tiles = ((pl.n_tiles + 1) / 2) * pl.m_tiles;
+    // Two weight tiles per CTA (512-row pair tiles) halve the activation
+    // bytes per MMA, when that still leaves a tile for every pair.
+    // The accumulators of a two-tile CTA are single-buffered (the epilogue
+    // stalls the MMAs once per tile), so this pays off only for long k.
+    const long long groups2 = (pl.n_tiles + 3) / 4;
+    pl.wt = (kPairWeightTiles == 2 && pl.k_steps >= kPairTwoTileMinSteps &&
+             groups2 * pl.m_tiles >= num_sms / 2) ? 2 : 1;
+    pl.tiles = ((pl.n_tiles + 2 * pl.wt - 1) / (2 * pl.wt)) * pl.m_tiles;
     pl.iters = pl.tiles * pl.units;
     pl.whole_tiles = 1;
-    pl.stage_bytes = pl.ks == 2 ? PairCfg<2>::stage_bytes(pl.bn) : PairCfg<1>::stage_bytes(pl.bn);
+    pl.stage_bytes = pl.ks * (pl.wt * kWTileBytes + (pl.bn / 2) * kStepK);
     pl.stages = kSmemBudget / pl.stage_bytes;
-    if (pl.stages > PairCfg<1>::kMaxStages) pl.stages = PairCfg<1>::kMaxStages;
-    pl.producers = kPlanProducers;
+    if (pl.stages > PairCfg<1, 1>::kMaxStages) pl.stages = PairCfg<1, 1>::kMaxStages;
+    pl.producers = producers_for(pl.stages);
     pl.smem_bytes = pair_smem_bytes(pl.stages, pl.stage_bytes);
     // The grid (pairs) is set at launch from the co-resident cluster count.
     pl.grid = 2 * static_cast<int>(pl.tiles < num_sms / 2 ? pl.tiles : num_sms / 2);
@@ -262,7 +280,7 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
   const int budget = kSmemBudget - pl.ra_bytes;
   pl.stages = budget / pl.stage_bytes;
   if (pl.stages > 16) pl.stages = 16;
-  pl.producers = kPlanProducers;
+  pl.producers = producers_for(pl.stages);
   pl.smem_bytes = linear_smem_bytes(pl.ra_bytes, pl.stages, pl.stage_bytes);
   if (pl.whole_tiles) {
     pl.grid = static_cast<int>(pl.tiles < num_sms ? pl.tiles : num_sms);
@@ -295,6 +313,24 @@ sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const Line
     }
   }
   return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), smem_bytes, st, ta, prm);
+}
+
+// Weight map for the pair kernel with two weight tiles per CTA: the packed
+// buffer as (256 B, 40, k steps, tiles), so that a box (256, 40, KS, 2) is
+// KS k steps of two consecutive tiles, landing as [tile][k step][10 KB].
+sfp8_status encode_weight_4d(CUtensorMap* map, const void* packed, uint64_t n_tiles,
+                             uint64_t k_steps, uint32_t box_steps) {
+  EncodeTiledFn enc = nullptr;
+  sfp8_status s = get_encoder(&enc);
+  if (s != SFP8_OK) return s;
+  cuuint64_t dims[4] = {256, kWTileBytes / 256, k_steps, n_tiles};
+  cuuint64_t strides[3] = {256, kWTileBytes, k_steps * kWTileBytes};
+  cuuint32_t box[4] = {256, kWTileBytes / 256, box_steps, 2};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(packed), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
 }
 
 // Weight map for the pair kernel: the packed buffer as (256 B, 40, tiles x
@@ -363,21 +399,23 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
 
 // CTA-pair GEMM: both maps, the co-resident pair count (queried once per
 // device), launch with programmatic stream serialisation.
-template <int KS>
-sfp8_status launch_pair_ks(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
-                           sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
-                           sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
-                           const void* bias, void* y, cudaStream_t st) {
-  auto kern = sparse_linear_pair_kernel<KS>;
+template <int KS, int WT>
+sfp8_status launch_pair_cfg(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
+                            sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
+                            sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
+                            const void* bias, void* y, cudaStream_t st) {
+  using Cfg = PairCfg<KS, WT>;
+  auto kern = sparse_linear_pair_kernel<KS, WT>;
+  constexpr int slot = (KS - 1) * 2 + (WT - 1);
   {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (dev->pair_clusters[KS] == 0) {
+    if (dev->pair_clusters[slot] == 0) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
           cudaSuccess)
         return SFP8_ERR_CUDA;
       cudaLaunchConfig_t qc{};
       qc.gridDim = dim3(2 * (dev->num_sms / 2));
-      qc.blockDim = dim3(kPairThreads);
+      qc.blockDim = dim3(Cfg::kThreads);
       qc.dynamicSmemBytes = kSmemLimit;
       cudaLaunchAttribute ca[1];
       ca[0].id = cudaLaunchAttributeClusterDimension;
@@ -391,17 +429,24 @@ sfp8_status launch_pair_ks(DeviceInfo* dev, const LinearPlan& pl, const void* a_
         cudaGetLastError();
         return SFP8_ERR_CUDA;
       }
-      dev->pair_clusters[KS] = clusters;
+      dev->pair_clusters[slot] = clusters;
     }
   }
-  CUtensorMap tw, ta;
+  CUtensorMap tw2, tw, ta;
   sfp8_status s = encode_weight_3d(&tw, packed, static_cast<uint64_t>(pl.n_tiles),
                                    static_cast<uint64_t>(pl.k_steps), KS);
   if (s != SFP8_OK) return s;
+  if (WT == 2) {
+    s = encode_weight_4d(&tw2, packed, static_cast<uint64_t>(pl.n_tiles),
+                         static_cast<uint64_t>(pl.k_steps), KS);
+    if (s != SFP8_OK) return s;
+  } else {
+    tw2 = tw;
+  }
   s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
                     static_cast<uint32_t>(pl.bn / 2), KS);
   if (s != SFP8_OK) return s;
-  const long long max_pairs = dev->pair_clusters[KS];
+  const long long max_pairs = dev->pair_clusters[slot];
   const int pairs = static_cast<int>(pl.tiles < max_pairs ? pl.tiles : max_pairs);
   PairParams prm{};
   prm.s_a = s_a;
@@ -412,7 +457,7 @@ sfp8_status launch_pair_ks(DeviceInfo* dev, const LinearPlan& pl, const void* a_
   prm.n = static_cast<int>(n);
   prm.k = static_cast<int>(k);
   prm.n_tiles = static_cast<int>(pl.n_tiles);
-  prm.n_pairs = static_cast<int>((pl.n_tiles + 1) / 2);
+  prm.n_groups = static_cast<int>((pl.n_tiles + 2 * WT - 1) / (2 * WT));
   prm.bn = pl.bn;
   prm.m_tiles = pl.m_tiles;
   prm.k_steps = pl.k_steps;
@@ -424,19 +469,30 @@ sfp8_status launch_pair_ks(DeviceInfo* dev, const LinearPlan& pl, const void* a_
   prm.producers = pl.producers;
   prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
                                 kPairTileN, static_cast<uint32_t>(pl.bn), true);
-  return launch_dependent(kern, dim3(2 * pairs), dim3(kPairThreads), pl.smem_bytes, st, tw, ta,
-                          prm);
+  return launch_dependent(kern, dim3(2 * pairs), dim3(Cfg::kThreads), pl.smem_bytes, st, tw2,
+                          tw, ta, prm);
 }
 
 sfp8_status launch_pair(DeviceInfo* dev, const LinearPlan& pl, const void* a_q,
                         sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
                         sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
                         const void* bias, void* y, cudaStream_t st) {
-  if (pl.ks == 2)
-    return launch_pair_ks<2>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
-                             st);
-  return launch_pair_ks<1>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
-                           st);
+  switch (pl.ks * 2 + pl.wt) {
+    case 1 * 2 + 1:
+      return launch_pair_cfg<1, 1>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k,
+                                   bias, y, st);
+    case 1 * 2 + 2:
+      return launch_pair_cfg<1, 2>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k,
+                                   bias, y, st);
+    case 2 * 2 + 1:
+      return launch_pair_cfg<2, 1>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k,
+                                   bias, y, st);
+    case 2 * 2 + 2:
+      return launch_pair_cfg<2, 2>(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k,
+                                   bias, y, st);
+    default:
+      return SFP8_ERR_UNSUPPORTED_SHAPE;   // no such plan is made
+  }
 }
 
 // Encodes the activation map and launches the GEMM for a validated plan.

@@ -26,7 +26,8 @@
 //               copies must come from several warps to overlap.
 //               With a single token tile (decode) the CTA's whole activation
 //               slice is loaded once instead (one 3-D TMA copy) and a stage is
-//               just the weight copy.
+//               just the weight copy; the weight beyond the first ring fill
+//               is prefetched into L2 at the start.
 //   warp 4      MMA issuer: per k step, copies the metadata block into tensor
 //               memory (tcgen05.cp 128x128b) and issues two 128 x BN x 64
 //               sparse MMAs; frees the stage with tcgen05.commit.
@@ -245,7 +246,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ producers
     // Lane 0 of producer warp w < P issues the copies of stages i with
     // i % P == w.
-    const int P = p.producers;
+    // no more producers than ring slots (see the host plan)
+    const int P = p.producers < S ? p.producers : S;
     const int pw = warp;
     if (lane == 0 && pw < P) {
       // A weight tile is read once when there is one token tile (decode:
@@ -279,6 +281,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (pre_count % P == pw) issue_weight(static_cast<int>(pre_count), t2, u);
             ++pre_count;
           }
+      }
+      if (pw == 0 && p.m_tiles == 1) {
+        // One token tile: everything past the stages just filled is read
+        // once, by this CTA.  Ask L2 to fetch it now, so that HBM keeps
+        // streaming while the ring waits for the activation.
+        const uint64_t pol_pf = l2_policy_evict_normal();
+        SegmentWalker pf(p, cta);
+        long long t3;
+        int b0, b1;
+        long long seen = 0;
+        while (pf.next(t3, b0, b1)) {
+          const int nt3 = static_cast<int>(t3 / p.m_tiles);
+          int s0 = b0;
+          if (seen < pre_count) {
+            const long long skip = pre_count - seen < b1 - b0 ? pre_count - seen : b1 - b0;
+            s0 = b0 + static_cast<int>(skip);
+          }
+          seen += b1 - b0;
+          if (s0 < b1) {
+            // a hint: at most the next 16 MB of the segment
+            long long bytes = static_cast<long long>(b1 - s0) * KS * kWTileBytes;
+            if (bytes > (16ll << 20)) bytes = 16ll << 20;
+            l2_prefetch_bulk(
+                p.packed + (static_cast<long long>(nt3) * p.k_steps + s0 * KS) * kWTileBytes,
+                static_cast<uint32_t>(bytes), pol_pf);
+          }
+        }
       }
       if (RA && pw == P - 1) {
         // The whole activation slice of this CTA, [k steps][BN rows][128 B],

@@ -23,17 +23,18 @@
 // takes N in steps of 32.)
 //
 // Roles (both CTAs unless noted):
-//   warps 0-3   producers: per stage, one TMA copy of KS packed weight tiles
-//               (a 3-D view of the 10 KB tiles) and one of the CTA's KS
-//               128-token activation tiles; all copies of a stage, both
-//               CTAs', complete on the stage barrier of rank 0, which rank 0
-//               arms with the byte count of the pair.
+//   warps 0-3   producers: per stage, one TMA copy of the CTA's packed
+//               weight tiles (a 3-D or 4-D view of the 10 KB tiles) and one
+//               of its activation tiles; all copies of a stage, both CTAs',
+//               complete on the stage barrier of rank 0, which rank 0 arms
+//               with the byte count of the pair.
 //   warp 4      rank 0: the MMA issuer (metadata copies and MMAs for the pair,
 //               commits multicast to both CTAs' barriers).  Rank 1: only
 //               allocates and frees tensor memory with rank 0.
-//   warps 5-12  epilogue: two warps per tensor-memory lane quadrant, each
-//               taking every other 16-column chunk of the accumulator:
-//               tensor memory -> registers -> scale/bias/bf16 -> global.
+//   warps 5-    epilogue: two warps per tensor-memory lane quadrant (and
+//               weight slot), each taking every other 16-column chunk of the
+//               accumulator: tensor memory -> registers -> scale/bias/bf16
+//               -> global.
 // Work split: tile t = n-pair * m_tiles + m-tile, pair p takes tiles p,
 // p + pairs, ...  No split-K.  Tensor memory: accumulator b at columns
 // [224 b, 224 b + BN), metadata of the stage's k steps at 448.
@@ -50,23 +51,30 @@
 
 namespace sfp8 {
 
-constexpr int kPairTileN = 256;        // weight rows per pair tile (MMA M)
+constexpr int kPairTileN = 256;        // weight rows per pair and weight slot (MMA M)
 constexpr int kPairMaxTokens = 224;    // largest BN: 2 x 224 + metadata <= 512
-constexpr int kPairEpiWarps = 8;
-constexpr int kPairEpiWarp0 = kProducerWarps + 1;
-constexpr int kPairThreads = 32 * (kProducerWarps + 1 + kPairEpiWarps);
+constexpr int kPairLoadWarps = kProducerWarps;
+constexpr int kPairMmaWarp = kPairLoadWarps;
+constexpr int kPairEpiWarp0 = kPairMmaWarp + 1;
 constexpr int kPairTmemCols = 512;
 constexpr int kPairMetaCol = 2 * kPairMaxTokens;  // after the two accumulators
 
-template <int KS>
+// KS k steps per stage; WT weight tiles (128 rows each) per CTA.
+//   WT = 1: pair tile 256 x BN, two accumulators (double buffer).
+//   WT = 2: pair tile 512 x BN, one accumulator per weight slot (single
+//           buffer): each activation byte loaded feeds twice the MMAs.
+template <int KS, int WT>
 struct PairCfg {
   static_assert(KS == 1 || KS == 2, "1 or 2 k steps per stage");
-  static constexpr int kWBytes = KS * kWTileBytes;
+  static_assert(WT == 1 || WT == 2, "1 or 2 weight tiles per CTA");
+  static constexpr int kWBytes = KS * WT * kWTileBytes;
   static constexpr int kMaxStages = 16;
-  static_assert(kPairMetaCol + 4 * KS <= kPairTmemCols, "metadata columns must fit");
+  static constexpr int kEpiWarps = 8 * WT;       // two per lane quadrant and slot
+  static constexpr int kThreads = 32 * (kPairLoadWarps + 1 + kEpiWarps);
+  static_assert(kPairMetaCol + 4 * KS * WT <= kPairTmemCols, "metadata columns must fit");
   // Shared memory of one stage for BN tokens per tile (a multiple of 1024).
   __host__ __device__ static constexpr int stage_bytes(int bn) {
-    return KS * (kWTileBytes + (bn / 2) * kStepK);
+    return KS * (WT * kWTileBytes + (bn / 2) * kStepK);
   }
 };
 
@@ -81,12 +89,12 @@ struct PairParams {
   __nv_bfloat16* y;
   int m, n, k;
   int n_tiles;      // 128-row weight tiles (ceil(n / 128))
-  int n_pairs;      // ceil(n_tiles / 2)
+  int n_groups;     // ceil(n_tiles / (2 WT)): weight-tile groups of a pair tile
   int bn;           // tokens per tile (multiple of 32, <= kPairMaxTokens)
   int m_tiles;      // ceil(m / bn)
   int k_steps;      // k / 128
   int units;        // stages per tile: k_steps / KS
-  int tiles;        // n_pairs * m_tiles
+  int tiles;        // n_groups * m_tiles
   int pairs;        // gridDim.x / 2
   int stages;
   int stage_bytes;  // PairCfg<KS>::stage_bytes(bn)
@@ -99,11 +107,12 @@ __device__ __forceinline__ void load_sa_pair(const PairParams& p, int m0, float 
   for (int j = 0; j < 16; ++j) sa[j] = (m0 + j < p.m) ? __ldg(p.s_a + m0 + j) : 0.0f;
 }
 
-template <int KS>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
-    sparse_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+template <int KS, int WT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kThreads, 1)
+    sparse_linear_pair_kernel(const __grid_constant__ CUtensorMap tm_w2,
+                              const __grid_constant__ CUtensorMap tm_w,
                               const __grid_constant__ CUtensorMap tm_a, const PairParams p) {
-  using Cfg = PairCfg<KS>;
+  using Cfg = PairCfg<KS, WT>;
   const int S = p.stages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -114,7 +123,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   constexpr int SM = Cfg::kMaxStages;
   uint64_t* full_bar = bars;                // [S], used on rank 0
   uint64_t* empty_bar = bars + SM;          // [S]
-  uint64_t* accf_bar = bars + 2 * SM;       // [2]
+  uint64_t* accf_bar = bars + 2 * SM;       // [2] (WT = 2 uses [0])
   uint64_t* acce_bar = bars + 2 * SM + 2;   // [2], rank 0
   uint64_t* drain_bar = bars + 2 * SM + 4;  // rank 0
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SM + 5);
@@ -135,17 +144,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&accf_bar[b]), 1);
-      mbar_init(smem_u32(&acce_bar[b]), 2 * kPairEpiWarps);
+      // every epilogue warp of both CTAs releases the accumulator(s)
+      mbar_init(smem_u32(&acce_bar[b]), 2 * Cfg::kEpiWarps);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
+    if (WT == 2) tma_prefetch_desc(&tm_w2);
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_a);
   }
-  if (warp == kMmaWarp) {
+  if (warp == kPairMmaWarp) {
     tmem_alloc_pair(smem_u32(tmem_slot), kPairTmemCols);
     tmem_relinquish_pair();
   }
@@ -155,24 +166,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < kProducerWarps) {
+  if (warp < kPairLoadWarps) {
     // ------------------------------------------------------------ producers
-    const int P = p.producers;
+    // no more producers than ring slots (see the host plan)
+    const int P = p.producers < S ? p.producers : S;
     const int pw = warp;
     if (lane == 0 && pw < P) {
       const uint64_t pol_w = l2_policy_evict_normal();
       const uint64_t pol_a = l2_policy_evict_last();
       auto full_of = [&](int stage) { return map_to_cta(smem_u32(&full_bar[stage]), 0); };
       auto issue_weight = [&](int stage, int tile, int u) {
-        const int np = tile / p.m_tiles;
-        int nt = 2 * np + static_cast<int>(rank);
-        // An odd tile count: rank 1 of the last pair re-reads the last tile
-        // (its rows are >= n and never stored).
-        if (nt >= p.n_tiles) nt = p.n_tiles - 1;
+        // CTA r holds weight tiles (2 WT) g + WT r + h, h < WT, of group g.
+        const int g = tile / p.m_tiles;
+        const int nt0 = 2 * WT * g + WT * static_cast<int>(rank);
+        const uint32_t dst = smem_u32(stage_base + stage * SB);
         // Rank 0 expects both CTAs' bytes of the stage.
         if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full_bar[stage]), 2 * SB);
-        tma_load_3d_pair(smem_u32(stage_base + stage * SB), &tm_w, 0, 0,
-                         nt * p.k_steps + u * KS, full_of(stage), pol_w);
+        if (WT == 2 && nt0 + 1 < p.n_tiles) {
+          // both tiles in one copy: box (256, 40, KS, 2) -> [h][j][10 KB]
+          tma_load_4d_pair(dst, &tm_w2, 0, 0, u * KS, nt0, full_of(stage), pol_w);
+        } else {
+#pragma unroll
+          for (int h = 0; h < WT; ++h) {
+            // Tiles past the end (a ragged last group) re-read the last tile;
+            // their rows are >= n and never stored.
+            int nt = nt0 + h;
+            if (nt >= p.n_tiles) nt = p.n_tiles - 1;
+            tma_load_3d_pair(dst + h * KS * kWTileBytes, &tm_w, 0, 0, nt * p.k_steps + u * KS,
+                             full_of(stage), pol_w);
+          }
+        }
       };
       auto issue_act = [&](int stage, int tile, int u) {
         const int mt = tile % p.m_tiles;
@@ -196,6 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (i % P != pw) continue;
           const int stage = static_cast<int>(i % S);
           if (i >= pre_count) {
+            // A ring slot is reused once the MMAs of its previous use are done.
             const uint32_t phase = static_cast<uint32_t>((i / S) & 1);
             if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag)) {
               ok = false;
@@ -217,7 +241,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kPairMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (rank == 0 && lane == 0) {
       grid_dependency_wait();
@@ -225,15 +249,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       const int a_tile_bytes = (p.bn / 2) * kStepK;
-      int acc = 0;
+      int acc = 0;              // WT = 1: accumulator buffer of this tile
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = pair; ok && t < p.tiles; t += p.pairs) {
-        // Accumulator `acc` is free once all 16 epilogue warps of the pair
-        // have read the tile before last.
+        // The accumulator(s) are free once every epilogue warp of the pair
+        // has read the tile that last used them.
         if (!mbar_wait_cluster(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kPairMaxTokens;
         for (int u = 0; u < p.units; ++u) {
           if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag)) {
             ok = false;
@@ -243,16 +266,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t st = smem_u32(stage_base + stage * SB);
 #pragma unroll
           for (int j = 0; j < KS; ++j) {
-            const uint32_t w_addr = st + j * kWTileBytes;
             const uint32_t a_addr = st + Cfg::kWBytes + j * a_tile_bytes;
-            tc_cp_128x128b_pair(e_tmem + 4 * j,
-                                smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t adesc = smem_desc(w_addr + 32 * h, 16, 512, kSwizzle64);
-              const uint64_t bdesc = smem_desc(a_addr + 64 * h, 16, 1024, kSwizzle128);
-              mma_sp_f8f6f4_pair(d_tmem, adesc, bdesc, e_tmem + 4 * j + 2 * h, p.idesc,
-                                 (u > 0 || j > 0 || h > 0) ? 1u : 0u);
+            for (int h = 0; h < WT; ++h) {
+              // weight slot h, k step j: [h][j][10 KB]
+              const uint32_t w_addr = st + (h * KS + j) * kWTileBytes;
+              const uint32_t e_col = e_tmem + 4 * (h * KS + j);
+              const uint32_t d_tmem = tmem_base + (WT == 1 ? acc : h) * kPairMaxTokens;
+              tc_cp_128x128b_pair(e_col, smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
+#pragma unroll
+              for (int kh = 0; kh < 2; ++kh) {
+                const uint64_t adesc = smem_desc(w_addr + 32 * kh, 16, 512, kSwizzle64);
+                const uint64_t bdesc = smem_desc(a_addr + 64 * kh, 16, 1024, kSwizzle128);
+                mma_sp_f8f6f4_pair(d_tmem, adesc, bdesc, e_col + 2 * kh, p.idesc,
+                                   (u > 0 || j > 0 || kh > 0) ? 1u : 0u);
+              }
             }
           }
           tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
@@ -263,8 +291,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         if (!ok) break;
         tc_commit_pair_mc(smem_u32(&accf_bar[acc]), 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (WT == 1) {
+          acc ^= 1;
+          if (acc == 0) acc_phase ^= 1u;
+        } else {
+          acc_phase ^= 1u;
+        }
       }
       tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
       volatile int no_abort = 0;
@@ -273,17 +305,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     grid_dependency_wait();
-    const int e = warp - kPairEpiWarp0;      // 0..7
+    const int e = warp - kPairEpiWarp0;      // 0 .. 8 WT - 1
     const int q = warp % 4;                   // tensor-memory lane quadrant
-    const int half = e / 4;                   // 16-column chunks half, half + 2, ...
+    const int half = (e / 4) % 2;             // 16-column chunks half, half + 2, ...
+    const int slot = e / 8;                   // weight slot (WT = 2)
     uint32_t acce_leader[2];
     for (int b = 0; b < 2; ++b) acce_leader[b] = map_to_cta(smem_u32(&acce_bar[b]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = pair; t < p.tiles; t += p.pairs) {
-      const int np = t / p.m_tiles;
+      const int g = t / p.m_tiles;
       const int mt = t % p.m_tiles;
-      const int n = (2 * np + static_cast<int>(rank)) * kTileN + q * 32 + lane;
+      const int nt = 2 * WT * g + WT * static_cast<int>(rank) + slot;
+      const int n = nt * kTileN + q * 32 + lane;
       const float sw = (n < p.n) ? __ldg(p.s_w + n) : 0.0f;
       const float bv = (p.bias != nullptr && n < p.n) ? __bfloat162float(p.bias[n]) : 0.0f;
       int ok = 1;
@@ -292,7 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                             static_cast<uint32_t>(acc * kPairMaxTokens);
+                             static_cast<uint32_t>((WT == 1 ? acc : slot) * kPairMaxTokens);
       const int m_tile0 = mt * p.bn;
 #pragma unroll 1
       for (int c = half; c < p.bn / 16; c += 2) {
@@ -314,8 +348,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader[acc]);
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (WT == 1) {
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      } else {
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -325,7 +363,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc_pair(tmem_base, kPairTmemCols);
+  if (warp == kPairMmaWarp) tmem_dealloc_pair(tmem_base, kPairTmemCols);
 }
 
 }  // namespace sfp8

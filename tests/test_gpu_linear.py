@@ -67,9 +67,11 @@ def test_ragged_multi_tile(m, k, n, pair):
 # Shapes for the CTA-pair kernel (512 tokens and more): an odd count of
 # 128-row weight tiles (the second CTA of the last pair has no rows), ragged
 # token tiles, a single k step, and token counts that choose different tile
-# widths (192, 224).
+# widths (192, 224).  The last four have enough tiles for two weight tiles
+# per CTA (512-row pair tiles), with a last group of 1, 2 or 4 valid tiles.
 PAIR_SHAPES = [(512, 128, 100), (700, 384, 390), (1000, 256, 1000), (2049, 128, 260),
-               (600, 640, 129)]
+               (600, 640, 129), (4000, 256, 2700), (4000, 256, 2600), (2049, 384, 5000),
+               (5000, 128, 1700)]
 
 
 @pytest.mark.parametrize("m,k,n", PAIR_SHAPES)
