@@ -46,9 +46,16 @@ K_DIM, N_DIM = 4096, 14336
 WEIGHT_COPIES = 8
 L2_NOTE = "rotating 8 copies of the compressed weight (8 x 36.7 MB > 126 MB L2)"
 
-# ncu DRAM traffic (read + write bytes) of one sparse-GEMM launch at M=16,
-# valid only for the kernel source it was measured on.
-NCU_TRAFFIC = {"sha1": None, "bytes_per_launch": None}
+# ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# sparse-GEMM launch, per (workload, M or shape), from the captures summarised
+# under profiles/; valid only while the kernel sources hash to `sha1`.
+KERNEL_SOURCES = ("device_common.cuh", "sparse_linear.cuh", "sparse_linear_pair.cuh")
+NCU_TRAFFIC = {
+    ("decode_gate_up_8b", 16): {"sha1": "b29457d6d6ae29bdb293ce8f0eba7d3f993a0a8b",
+                                "bytes_per_launch": 36888320},
+    ("prefill_8b", 2): {"sha1": "b29457d6d6ae29bdb293ce8f0eba7d3f993a0a8b",
+                        "bytes_per_launch": 271275264},
+}
 
 
 def compressed_weight_bytes(n, k):
@@ -63,9 +70,12 @@ def gemm_algorithmic_bytes(m, n, k):
 
 
 def kernel_source_sha1():
-    p = os.path.join(ROOT, "semi_structured_sparse_rowwise_b200", "csrc", "sparse_linear.cuh")
-    with open(p, "rb") as f:
-        return hashlib.sha1(f.read()).hexdigest()
+    h = hashlib.sha1()
+    for name in KERNEL_SOURCES:
+        p = os.path.join(ROOT, "semi_structured_sparse_rowwise_b200", "csrc", name)
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def measured_peaks():
@@ -404,8 +414,9 @@ def run_ours(args):
         peak, peak_kind = measured_tensor_peak()
         achieved = flops / (gemm_us * 1e-6) / 1e12
     traffic = None
-    if NCU_TRAFFIC["sha1"] == kernel_source_sha1():
-        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    rec = NCU_TRAFFIC.get((args.workload, args.shape if prefill else m))
+    if rec is not None and rec["sha1"] == kernel_source_sha1():
+        traffic = rec["bytes_per_launch"]
 
     # ---- end to end through the layer, host buffers, eager calls
     layer = S.SparseFp8Linear.from_compressed(copies[0][0], copies[0][1], n, k)
@@ -475,7 +486,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor" if prefill else "hbm", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s" if prefill else "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "sparse_linear_kernel",
+                     "kernel": "sparse_linear_pair_kernel" if m >= 512 else "sparse_linear_kernel",
                      "algorithmic_bytes_per_launch": alg,
                      "algorithmic_flop_per_launch": flops, "us_per_launch": gemm_us,
                      "peak_source": peak_kind},

@@ -218,8 +218,9 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
  *    workspace.
  *  - Size limit: problems whose sfp8_sparse_linear_workspace_bytes(m, n, k)
  *    exceeds SFP8_NOALLOC_SCRATCH_BYTES are rejected with SFP8_ERR_WORKSPACE
- *    before anything is launched (on a 148-SM B200 this admits m <= 32 for
- *    any n and k).
+ *    before anything is launched (on a 148-SM B200 this admits any n and k
+ *    for m <= 32 and for m >= 512, which need at most 4.8 MB and no scratch;
+ *    between them it depends on the work split chosen for n and k).
  *  - The first call on a device looks up the buffer's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    outside any stream capture.
