@@ -3,12 +3,21 @@
 // scaling of its title and item 1, the dynamic-activation path of item 4).
 //
 // Per row: amax = max |x| (fp32), s = max(amax, 1e-12f) / FP8_MAX (IEEE fp32
-// division), q = cvt.rn.satfinite(x / s) with an IEEE fp32 division per
-// element.  One HBM read of x: each group of TPR threads holds its whole row
-// in registers (CHUNKS 16-byte vectors per thread), reduces the row amax
-// with warp shuffles (and shared memory across warps when TPR > 32), then
-// converts from the registers.  Rows too long for the register tile use a
-// two-sweep variant that re-reads the row (from L2).
+// division), q = cvt.rn.satfinite(x / s) where x / s is the correctly rounded
+// fp32 quotient.  One HBM read of x: each group of TPR threads holds its
+// whole row in registers (CHUNKS 16-byte vectors per thread), reduces the row
+// amax with warp shuffles (and shared memory across warps when TPR > 32),
+// then converts from the registers.  Rows too long for the register tile use
+// a two-sweep variant that re-reads the row (from L2).
+//
+// The quotient without a division per element: t = x * r with r = 1/s
+// correctly rounded is within 3 units in the last place of the correctly
+// rounded x / s (two roundings of relative size <= 2^-24 each, then the
+// quotient's own rounding).  FP8 rounding is monotone, so t and x / s give
+// the same code unless an FP8 rounding midpoint lies within those 3 units of
+// t; when t is within 4 units of a midpoint (or in the FP8 subnormal range,
+// where the rounding position moves), the quotient is computed by an IEEE
+// division instead.  The codes are therefore exactly those of x / s.
 //
 // The kernels are launched as programmatic dependents: they let their own
 // dependents (the GEMM) launch at once, then wait for the preceding grid to
@@ -26,6 +35,9 @@ namespace sfp8 {
 
 template <typename T>
 struct InputTraits;
+// Per input type: widening of one 16-byte vector to floats, and the vector's
+// max |value| folded into a running amax.  The 16-bit types take the max on
+// packed pairs (exact: the max of the values, widened once).
 template <>
 struct InputTraits<__nv_bfloat16> {
   static constexpr int kPerVec = 8;
@@ -37,6 +49,12 @@ struct InputTraits<__nv_bfloat16> {
       f[2 * i] = t.x;
       f[2 * i + 1] = t.y;
     }
+  }
+  __device__ static float abs_max(const uint4& v, float amax) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const __nv_bfloat162 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])),
+                                     __hmax2(__habs2(h[2]), __habs2(h[3])));
+    return fmaxf(amax, fmaxf(__low2float(m), __high2float(m)));
   }
 };
 template <>
@@ -51,6 +69,12 @@ struct InputTraits<__half> {
       f[2 * i + 1] = t.y;
     }
   }
+  __device__ static float abs_max(const uint4& v, float amax) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+    const __half2 m = __hmax2(__hmax2(__habs2(h[0]), __habs2(h[1])),
+                              __hmax2(__habs2(h[2]), __habs2(h[3])));
+    return fmaxf(amax, fmaxf(__low2float(m), __high2float(m)));
+  }
 };
 template <>
 struct InputTraits<float> {
@@ -60,6 +84,10 @@ struct InputTraits<float> {
     f[1] = __uint_as_float(v.y);
     f[2] = __uint_as_float(v.z);
     f[3] = __uint_as_float(v.w);
+  }
+  __device__ static float abs_max(const uint4& v, float amax) {
+    return fmaxf(fmaxf(amax, fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y)))),
+                 fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
   }
 };
 
@@ -86,18 +114,42 @@ __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi) {
       __nv_cvt_float2_to_fp8x2(v, __NV_SATFINITE, Fp8Out<kFmt>::kInterp));
 }
 
+// True when the FP8 code of every fp32 value within 4 units in the last
+// place of t equals the code of t: |t| is at least the smallest normal FP8
+// value and t's bits below the FP8 mantissa are more than 4 away from the
+// half-way pattern (or t is zero).
+template <int kFmt>
+__device__ __forceinline__ bool fp8_rounding_is_clear(float t) {
+  constexpr int kMant = kFmt == SFP8_E4M3 ? 3 : 2;          // FP8 mantissa bits
+  constexpr int kEmin = kFmt == SFP8_E4M3 ? -6 : -14;        // smallest normal exponent
+  constexpr uint32_t kMinNormal = static_cast<uint32_t>(127 + kEmin) << 23;
+  constexpr int kDrop = 23 - kMant;                          // fp32 bits rounded away
+  constexpr uint32_t kHalf = 1u << (kDrop - 1);
+  const uint32_t u = __float_as_uint(t) & 0x7FFFFFFFu;
+  // (rem - half + 4) mod 2^32 > 8  <=>  |rem - half| > 4
+  const uint32_t d = (u & ((1u << kDrop) - 1u)) - kHalf + 4u;
+  return (u >= kMinNormal && d > 8u) || u == 0u;
+}
+
 // Quantises one 16-byte input vector (already widened to floats) into
-// kPerVec codes packed little-endian.
+// kPerVec codes packed little-endian; s is the row scale, r = 1/s.
 template <int kFmt, int kPerVec>
-__device__ __forceinline__ void quantize_vec(const float (&f)[kPerVec], float s,
+__device__ __forceinline__ void quantize_vec(const float (&f)[kPerVec], float s, float r,
                                              uint32_t (&out)[kPerVec / 4]) {
 #pragma unroll
   for (int w = 0; w < kPerVec / 4; ++w) {
-    const float a = __fdiv_rn(f[4 * w + 0], s);
-    const float b = __fdiv_rn(f[4 * w + 1], s);
-    const float c = __fdiv_rn(f[4 * w + 2], s);
-    const float d = __fdiv_rn(f[4 * w + 3], s);
-    out[w] = cvt_pair<kFmt>(a, b) | (cvt_pair<kFmt>(c, d) << 16);
+    float t[4];
+    bool clear = true;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      t[i] = __fmul_rn(f[4 * w + i], r);
+      clear = clear && fp8_rounding_is_clear<kFmt>(t[i]);
+    }
+    if (!clear) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[i] = __fdiv_rn(f[4 * w + i], s);
+    }
+    out[w] = cvt_pair<kFmt>(t[0], t[1]) | (cvt_pair<kFmt>(t[2], t[3]) << 16);
   }
 }
 
@@ -158,14 +210,12 @@ __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
     const int64_t vi = static_cast<int64_t>(c) * TPR + t;
     if (row_ok && vi < nvec) {
       v[c] = __ldg(reinterpret_cast<const uint4*>(xr + vi * P));
-      float f[P];
-      Tr::to_float(v[c], f);
-#pragma unroll
-      for (int i = 0; i < P; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      amax = Tr::abs_max(v[c], amax);
     }
   }
   amax = row_group_max<TPR>(amax, red);
   const float s = __fdiv_rn(fmaxf(amax, kGuardAmax), Fp8Out<kFmt>::kMax);
+  const float r = __frcp_rn(s);
   if (!row_ok) return;
   if (t == 0) scales[row] = s;
   uint8_t* qr = q + row * cols;
@@ -176,8 +226,94 @@ __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
       float f[P];
       Tr::to_float(v[c], f);
       uint32_t w[P / 4];
-      quantize_vec<kFmt, P>(f, s, w);
+      quantize_vec<kFmt, P>(f, s, r, w);
       store_codes<P>(qr + vi * P, w);
+    }
+  }
+}
+
+// Streaming quantiser for rows of up to 48 KB: one persistent CTA per SM.
+// Lane 0 of warp 0 streams the CTA's rows (rows b, b + grid, ...) into a
+// ring of `slots` shared-memory row buffers, one bulk copy per row; consumer
+// warp c (of `consumers`) owns ring slots c, c + consumers, ... (slots is a
+// multiple of consumers, so every slot has one consumer and no wait can run
+// two phases ahead).  A consumer reads its row from shared memory twice
+// (amax, then convert) and writes the codes straight to global memory.  The
+// ring keeps slots x row bytes in flight per SM whatever the registers.
+constexpr int kQuantMaxConsumers = 24;
+constexpr int kQuantMaxSlots = 24;
+constexpr int kQuantThreads = 32 * (1 + kQuantMaxConsumers);
+
+template <typename T, int kFmt>
+__global__ void __launch_bounds__(kQuantThreads, 1)
+    quantize_rowwise_stream_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
+                                   int64_t ld, uint8_t* __restrict__ q,
+                                   float* __restrict__ scales, int slots, int consumers) {
+  grid_dependents_launch();
+  using Tr = InputTraits<T>;
+  constexpr int P = Tr::kPerVec;
+  extern __shared__ __align__(128) uint8_t qsmem[];
+  const int row_bytes = static_cast<int>(cols) * static_cast<int>(sizeof(T));
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsmem + static_cast<size_t>(slots) * row_bytes);
+  uint64_t* empty = full + kQuantMaxSlots;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kQuantMaxSlots);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < slots; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  grid_dependency_wait();
+  const int64_t my_rows = rows > blockIdx.x ? (rows - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_first();
+      for (int64_t j = 0; j < my_rows; ++j) {
+        const int slot = static_cast<int>(j % slots);
+        if (j >= slots &&
+            !mbar_wait(smem_u32(&empty[slot]), static_cast<uint32_t>(((j / slots) - 1) & 1),
+                       abort_flag))
+          break;
+        const int64_t row = blockIdx.x + j * gridDim.x;
+        mbar_arrive_expect_tx(smem_u32(&full[slot]), row_bytes);
+        bulk_load(smem_u32(qsmem + static_cast<size_t>(slot) * row_bytes), x + row * ld,
+                  row_bytes, smem_u32(&full[slot]), pol);
+      }
+    }
+  } else if (warp - 1 < consumers) {
+    const int c = warp - 1;
+    const int nvec = static_cast<int>(cols) / P;
+    for (int64_t j = c; j < my_rows; j += consumers) {
+      const int slot = static_cast<int>(j % slots);
+      // every lane waits: the barrier's completion is what makes the copied
+      // row visible to the lane that reads it
+      const bool ok =
+          mbar_wait(smem_u32(&full[slot]), static_cast<uint32_t>((j / slots) & 1), abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint4* src = reinterpret_cast<const uint4*>(qsmem + static_cast<size_t>(slot) * row_bytes);
+      float amax = 0.0f;
+      for (int vi = lane; vi < nvec; vi += 32) amax = Tr::abs_max(src[vi], amax);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = __fdiv_rn(fmaxf(amax, kGuardAmax), Fp8Out<kFmt>::kMax);
+      const float r = __frcp_rn(s);
+      const int64_t row = blockIdx.x + j * gridDim.x;
+      if (lane == 0) scales[row] = s;
+      uint8_t* qr = q + row * cols;
+      for (int vi = lane; vi < nvec; vi += 32) {
+        float f[P];
+        Tr::to_float(src[vi], f);
+        uint32_t w[P / 4];
+        quantize_vec<kFmt, P>(f, s, r, w);
+        store_codes<P>(qr + static_cast<int64_t>(vi) * P, w);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
     }
   }
 }
@@ -198,14 +334,11 @@ __global__ void __launch_bounds__(1024)
   const int64_t nvec = cols / P;
   float amax = 0.0f;
   for (int64_t vi = threadIdx.x; vi < nvec; vi += blockDim.x) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(xr + vi * P));
-    float f[P];
-    Tr::to_float(v, f);
-#pragma unroll
-    for (int i = 0; i < P; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = Tr::abs_max(__ldg(reinterpret_cast<const uint4*>(xr + vi * P)), amax);
   }
   amax = row_group_max<1024>(amax, red);
   const float s = __fdiv_rn(fmaxf(amax, kGuardAmax), Fp8Out<kFmt>::kMax);
+  const float r = __frcp_rn(s);
   if (threadIdx.x == 0) scales[row] = s;
   uint8_t* qr = q + row * cols;
   for (int64_t vi = threadIdx.x; vi < nvec; vi += blockDim.x) {
@@ -213,7 +346,7 @@ __global__ void __launch_bounds__(1024)
     float f[P];
     Tr::to_float(v, f);
     uint32_t w[P / 4];
-    quantize_vec<kFmt, P>(f, s, w);
+    quantize_vec<kFmt, P>(f, s, r, w);
     store_codes<P>(qr + vi * P, w);
   }
 }

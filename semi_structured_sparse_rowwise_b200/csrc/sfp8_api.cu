@@ -122,7 +122,15 @@ sfp8_status launch_dependent(Kernel kern, dim3 grid, dim3 block, size_t smem, cu
   return SFP8_OK;
 }
 
+constexpr int kSmemLimit = 232448;                 // 227 KB: largest dynamic smem per CTA
+
 // ------------------------------------------------------------------ quantise
+
+// Row count from which the streaming quantiser is used (below it, a few
+// register-tile blocks finish sooner).
+constexpr int64_t kQuantStreamMinRows = 256;
+constexpr int kQuantRingSlots = 24;         // <= kQuantMaxSlots
+constexpr int kQuantSlotsPerConsumer = 1;   // consumers <= kQuantMaxConsumers
 
 template <typename T, int kFmt>
 sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
@@ -136,19 +144,51 @@ sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
   }
   constexpr int P = InputTraits<T>::kPerVec;
   const int64_t nvec = cols / P;
-  constexpr int kChunks = 8;
-  if (nvec <= 32 * kChunks) {
+  // Many rows of up to 16 KB: the streaming kernel (one CTA per SM, a ring
+  // of row buffers filled by bulk copies; measured faster than the register
+  // tiles up to 16 KB rows, slower beyond).
+  const int64_t row_bytes = cols * static_cast<int64_t>(sizeof(T));
+  if (rows >= kQuantStreamMinRows && row_bytes <= 16 * 1024) {
+    DeviceInfo* dev = nullptr;
+    sfp8_status s = current_device(&dev);
+    if (s != SFP8_OK) return s;
+    // Ring: up to 192 KB of rows in flight; every consumer warp owns
+    // slots / consumers ring slots (a whole number).
+    int slots = static_cast<int>((192 * 1024) / row_bytes);
+    if (slots > kQuantRingSlots) slots = kQuantRingSlots;
+    int consumers = slots / kQuantSlotsPerConsumer;
+    if (consumers < 1) consumers = 1;
+    slots = consumers * kQuantSlotsPerConsumer;
+    const int smem = static_cast<int>(slots * row_bytes) + 1024;
+    auto kern = quantize_rowwise_stream_kernel<T, kFmt>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) !=
+        cudaSuccess)
+      return SFP8_ERR_CUDA;
+    const int64_t grid = rows < dev->num_sms ? rows : dev->num_sms;
+    return launch_dependent(kern, dim3(static_cast<unsigned>(grid)), dim3(kQuantThreads),
+                            static_cast<size_t>(smem), st, xp, rows, cols, ld, qp, scales, slots,
+                            consumers);
+  }
+  // Rows in registers: one warp per row up to 512 vectors (16 per lane:
+  // 8 KB of bf16 in flight per warp), then 4 and 16 warps per row (the 16-warp
+  // tile holds 8 vectors per thread: 16 would not fit 512 threads' registers).
+  if (nvec <= 32 * 4) {
     const int64_t blocks = (rows + 7) / 8;
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, kChunks>,
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, 4>,
                             dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
                             ld, qp, scales);
-  } else if (nvec <= 128 * kChunks) {
+  } else if (nvec <= 32 * 16) {
+    const int64_t blocks = (rows + 7) / 8;
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, 16>,
+                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
+                            ld, qp, scales);
+  } else if (nvec <= 128 * 16) {
     const int64_t blocks = (rows + 1) / 2;
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 128, kChunks>,
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 128, 16>,
                             dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
                             ld, qp, scales);
-  } else if (nvec <= 512 * kChunks) {
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 512, kChunks>,
+  } else if (nvec <= 512 * 8) {
+    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 512, 8>,
                             dim3(static_cast<unsigned>(rows)), dim3(512), 0, st, xp, rows, cols,
                             ld, qp, scales);
   }
@@ -166,7 +206,6 @@ sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64
 
 // ------------------------------------------------------------------ linear plan
 
-constexpr int kSmemLimit = 232448;                 // 227 KB: largest dynamic smem per CTA
 constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice limit
 constexpr int kPlanProducers = 4;                  // producer warps used
 

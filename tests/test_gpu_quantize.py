@@ -42,6 +42,72 @@ def test_exhaustive_bf16_sweep(fmt):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("fmt,amax", [("e4m3", 300.0), ("e5m2", 39936.0)])
+def test_exhaustive_bf16_sweep_scaled(fmt, amax):
+    """Every finite bf16 value up to amax in rows whose amax is not FP8_MAX times
+    a power of two, so s = amax / FP8_MAX is inexact and the quotients land all
+    over the FP8 grid (midpoints included)."""
+    mx = np.float32(amax)
+    v = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32)
+    v = v[np.isfinite(v) & (np.abs(v) <= mx)]
+    width = 256
+    v = np.concatenate([v, np.zeros((-v.size) % (width - 1), np.float32)])
+    body = v.reshape(-1, width - 1)
+    x = np.concatenate([np.full((body.shape[0], 1), mx, np.float32), body], axis=1)
+    xd = _to_dev(x, torch.bfloat16)
+    q, s = S.sfp8_quantize_rowwise(xd, fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def _near_midpoint_rows(fmt, seed, n_rows):
+    """fp32 rows whose quotients x / s fall within a few units in the last
+    place of FP8 rounding midpoints (and on both sides of them)."""
+    rng = np.random.default_rng(seed)
+    table = oracle.decode_table(fmt)
+    pos = np.unique(table[np.isfinite(table) & (table >= 0)])
+    mids = (pos[:-1] + pos[1:]) / 2.0
+    fmax = np.float32(oracle.fp8_max(fmt))
+    rows = []
+    for _ in range(n_rows):
+        amax = np.float32(rng.uniform(0.5, 3.0) * 2.0 ** int(rng.integers(-20, 20)))
+        s = np.float32(amax / fmax)
+        base = (mids * np.float64(s)).astype(np.float32)
+        cands = [base]
+        up, dn = base.copy(), base.copy()
+        for _ in range(5):
+            up = np.nextafter(up, np.float32(np.inf))
+            dn = np.nextafter(dn, np.float32(0.0))
+            cands += [up.copy(), dn.copy()]
+        v = np.concatenate(cands)
+        v = v[np.abs(v) <= amax]
+        rows.append(np.concatenate([[amax], v, -v]).astype(np.float32))
+    width = (max(r.size for r in rows) + 15) // 16 * 16
+    x = np.zeros((len(rows), width), np.float32)
+    for i, r in enumerate(rows):
+        x[i, :r.size] = r
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_near_midpoint_quotients(fmt):
+    """The quantiser's division-free path must hand every quotient near an FP8
+    rounding midpoint to an exact division: codes equal the oracle's (IEEE
+    fp32 division, then one rounding) bit for bit."""
+    x = _near_midpoint_rows(fmt, 77 if fmt == "e4m3" else 78, 48)
+    q, s = S.sfp8_quantize_rowwise(_to_dev(x, torch.float32), fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    # the rows do exercise the near-midpoint case: quotients that a 1-ulp
+    # error would round differently
+    quo = x / s_ref[:, None]
+    up = oracle.encode_rne_sat(np.nextafter(quo, np.float32(np.inf)), fmt)
+    dn = oracle.encode_rne_sat(np.nextafter(quo, np.float32(-np.inf)), fmt)
+    assert int((up != dn).sum()) > 1000
+
+
 CASES = [
     # rows, cols, torch dtype, distribution
     (16, 128, torch.bfloat16, "normal"),
@@ -80,6 +146,27 @@ def test_strided_input(fmt):
     xd = wide[:, 128:384]                  # ld = 512, cols = 256
     q, s = S.sfp8_quantize_rowwise(xd, fmt)
     q_ref, s_ref = oracle.quantize_rowwise(oracle.bf16_bits_to_f32(bits)[:, 128:384], fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("rows,cols,ld,dtype", [(300, 256, 512, torch.bfloat16),
+                                                (257, 16, 16, torch.bfloat16),
+                                                (600, 4096, 4096, torch.float32),
+                                                (1000, 8192, 8192, torch.bfloat16),
+                                                (700, 6144, 6144, torch.bfloat16)])
+def test_streaming_quantiser_shapes(rows, cols, ld, dtype, fmt):
+    """Row counts that use the streaming quantiser (one CTA per SM, ring of row
+    buffers): strided rows, 32-byte rows, 16 KB rows, ring sizes of 24 and 16
+    slots, rows not a multiple of the grid."""
+    bits = synthetic.activation(5150 + rows + cols, rows, ld, dist="student_t3", zero_row_frac=0.05)
+    x32 = oracle.bf16_bits_to_f32(bits)
+    wide = _to_dev(x32, dtype)
+    xd = wide[:, :cols]
+    xr = _ref_from_dev(xd)
+    q, s = S.sfp8_quantize_rowwise(xd, fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(xr, fmt)
     assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
