@@ -169,28 +169,31 @@ sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
                             static_cast<size_t>(smem), st, xp, rows, cols, ld, qp, scales, slots,
                             consumers);
   }
-  // Rows in registers: one warp per row up to 512 vectors (16 per lane:
-  // 8 KB of bf16 in flight per warp), then 4 and 16 warps per row (the 16-warp
-  // tile holds 8 vectors per thread: 16 would not fit 512 threads' registers).
-  if (nvec <= 32 * 4) {
-    const int64_t blocks = (rows + 7) / 8;
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, 4>,
-                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
-                            ld, qp, scales);
-  } else if (nvec <= 32 * 16) {
-    const int64_t blocks = (rows + 7) / 8;
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 32, 16>,
-                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
-                            ld, qp, scales);
-  } else if (nvec <= 128 * 16) {
-    const int64_t blocks = (rows + 1) / 2;
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 128, 16>,
-                            dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, xp, rows, cols,
-                            ld, qp, scales);
-  } else if (nvec <= 512 * 8) {
-    return launch_dependent(quantize_rowwise_kernel<T, kFmt, 512, 8>,
-                            dim3(static_cast<unsigned>(rows)), dim3(512), 0, st, xp, rows, cols,
-                            ld, qp, scales);
+  // Rows in registers.  Few rows (a decode step): as many threads per row as
+  // the row has vectors (up to 512), so each thread converts one to eight
+  // vectors and the call is short.  Many long rows: one warp per row up to
+  // 512 vectors (16 per lane: 8 KB of bf16 in flight per warp), then 4 and
+  // 16 warps per row (the 16-warp tile holds 8 vectors per thread: 16 would
+  // not fit 512 threads' registers).
+  auto launch = [&](auto kern, int tpr) {
+    const int threads = tpr > 256 ? tpr : 256;
+    const int64_t per_block = threads / tpr;
+    const int64_t blocks = (rows + per_block - 1) / per_block;
+    return launch_dependent(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, st, xp,
+                            rows, cols, ld, qp, scales);
+  };
+  if (rows < kQuantStreamMinRows) {
+    if (nvec <= 32) return launch(quantize_rowwise_kernel<T, kFmt, 32, 1>, 32);
+    if (nvec <= 128) return launch(quantize_rowwise_kernel<T, kFmt, 128, 1>, 128);
+    if (nvec <= 512) return launch(quantize_rowwise_kernel<T, kFmt, 512, 1>, 512);
+    if (nvec <= 1024) return launch(quantize_rowwise_kernel<T, kFmt, 512, 2>, 512);
+    if (nvec <= 2048) return launch(quantize_rowwise_kernel<T, kFmt, 512, 4>, 512);
+    if (nvec <= 4096) return launch(quantize_rowwise_kernel<T, kFmt, 512, 8>, 512);
+  } else {
+    if (nvec <= 32 * 4) return launch(quantize_rowwise_kernel<T, kFmt, 32, 4>, 32);
+    if (nvec <= 32 * 16) return launch(quantize_rowwise_kernel<T, kFmt, 32, 16>, 32);
+    if (nvec <= 128 * 16) return launch(quantize_rowwise_kernel<T, kFmt, 128, 16>, 128);
+    if (nvec <= 512 * 8) return launch(quantize_rowwise_kernel<T, kFmt, 512, 8>, 512);
   }
   return launch_dependent(quantize_rowwise_long_kernel<T, kFmt>,
                           dim3(static_cast<unsigned>(rows)), dim3(1024), 0, st, xp, rows, cols,
