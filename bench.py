@@ -69,6 +69,7 @@ def gemm_algorithmic_bytes(m, n, k):
     return compressed_weight_bytes(n, k) + 4 * n + m * k + 4 * m + 2 * m * n
 
 
+
 def kernel_source_sha1():
     h = hashlib.sha1()
     for name in KERNEL_SOURCES:
@@ -341,6 +342,7 @@ def run_ours(args):
     ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev)
           for _ in range(WEIGHT_COPIES if not prefill else 2)]
     ws = S.new_workspace(m, n, k, dev)
+    ws_q = S.new_quant_workspace(m, n, k, dev)
 
     def quantize():
         S.sfp8_quantize_rowwise(x_dev, "e4m3", q=aq, scales=sa)
@@ -351,8 +353,10 @@ def run_ours(args):
                              workspace=ws)
 
     def step(j):
-        quantize()
-        gemm(j)
+        # one forward of the layer: one library call (quantiser + GEMM kernels)
+        pk, s = copies[j % len(copies)]
+        S.sfp8_sparse_linear_quant(x_dev, "e4m3", pk, "e4m3", s, n, k, out=ys[j % len(ys)],
+                                   workspace=ws_q, a_q=aq, s_a=sa)
 
     for j in range(args.warmup):
         step(j)
@@ -408,8 +412,10 @@ def run_ours(args):
     g_q.replay()
     ms_q = dist_max(timed(g_q), world, dev)
     peak, peak_kind = measured_peaks()
+    # the dominant kernel of the step: the GEMM
+    kernel_us = gemm_us
     alg = gemm_algorithmic_bytes(m, n, k)
-    achieved = alg / (gemm_us * 1e-6) / 1e9
+    achieved = alg / (kernel_us * 1e-6) / 1e9
     if prefill:
         peak, peak_kind = measured_tensor_peak()
         achieved = flops / (gemm_us * 1e-6) / 1e12
@@ -480,15 +486,16 @@ def run_ours(args):
                    "rotating %d weight copies; every step's weight is evicted from L2 by the "
                    "others (%d x %.1f MB + activations and outputs > 126 MB)"
                    % (len(copies), len(copies), wbytes / 1e6),
-                   "step": "sfp8_quantize_rowwise + sfp8_sparse_linear",
+                   "step": "sfp8_sparse_linear_quant (quantiser + GEMM kernels)",
                    "weight_bytes_per_step": wbytes, "seeds": seeds,
                    "parallelism": "replica" if world > 1 else "single"},
         "roofline": {"bound": "tensor" if prefill else "hbm", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s" if prefill else "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "sparse_linear_pair_kernel" if m >= 512 else "sparse_linear_kernel",
+                     "kernel": ("sparse_linear_pair_kernel" if m >= 512 else
+                                "sparse_linear_kernel"),
                      "algorithmic_bytes_per_launch": alg,
-                     "algorithmic_flop_per_launch": flops, "us_per_launch": gemm_us,
+                     "algorithmic_flop_per_launch": flops, "us_per_launch": kernel_us,
                      "peak_source": peak_kind},
         "quantize_us_per_launch": ms_q * 1e3 / steps,
         "e2e": e2e,

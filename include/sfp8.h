@@ -196,6 +196,40 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace for sfp8_sparse_linear_quant (the same as sfp8_sparse_linear's
+ * for these sizes).
+ */
+size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/*
+ * The layer's forward in one call: dynamic row-wise quantisation of the
+ * activation (exactly sfp8_quantize_rowwise: page "Add CUTLASS-based
+ * row-wise scaled sparse FP8 kernel", items 1 and 4) followed by the sparse
+ * linear (exactly sfp8_sparse_linear), both launched on `stream` (the GEMM
+ * as a programmatic dependent of the quantiser, so its weight stream starts
+ * while the activation is being quantised).
+ *
+ *  x       device, [m, ld_x] bf16 / fp16 / fp32 activation, 16-byte aligned,
+ *          ld_x >= k, ld_x * element size a multiple of 16.
+ *  a_dtype SFP8_E4M3 or SFP8_E5M2: the activation's FP8 format.
+ *  a_q     device, [m, k] u8, written (the quantised activation).
+ *  s_a     device, [m] float32, written (its row scales).
+ *  packed, w_dtype, s_w, n, k, bias, y: as for sfp8_sparse_linear.
+ *  workspace  >= sfp8_sparse_linear_quant_workspace_bytes(m, n, k) bytes,
+ *          zero before the first call (left zero by every call).
+ *
+ * Returns the first failing status of the two steps (validation of both
+ * before anything is launched where the arguments allow).  With n == 0 only
+ * the activation is quantised.
+ */
+sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
+                                     sfp8_dtype a_dtype, void* a_q, float* s_a, int64_t m,
+                                     const void* packed, sfp8_dtype w_dtype,
+                                     const float* s_w, int64_t n, int64_t k,
+                                     const void* bias, void* y, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * Size of the scratch buffer built into the library for
  * sfp8_sparse_linear_noalloc (per device that loads the library).
  */

@@ -11,7 +11,8 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_compress_24, sfp8_decompress_24,
                       sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
                       sfp8_sparse_linear, sfp8_sparse_linear_noalloc,
-                      sfp8_read_device_status,
+                      sfp8_sparse_linear_quant, sfp8_sparse_linear_quant_workspace_bytes,
+                      new_quant_workspace, sfp8_read_device_status,
                       sfp8_status_string, sfp8_layout_version)
 from .layer import SparseFp8Linear
 
@@ -21,6 +22,8 @@ __all__ = [
     "sfp8_compressed_bytes",
     "sfp8_compress_24", "sfp8_decompress_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
-    "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_read_device_status", "sfp8_status_string",
+    "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_sparse_linear_quant",
+    "sfp8_sparse_linear_quant_workspace_bytes", "new_quant_workspace",
+    "sfp8_read_device_status", "sfp8_status_string",
     "sfp8_layout_version", "SparseFp8Linear",
 ]

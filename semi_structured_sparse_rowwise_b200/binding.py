@@ -46,6 +46,10 @@ SIGNATURES = {
     "sfp8_sparse_linear_noalloc": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p,
                                           _i32, _c_void_p, _i64, _i64, _c_void_p,
                                           _c_void_p, _c_void_p]),
+    "sfp8_sparse_linear_quant_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "sfp8_sparse_linear_quant": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p, _c_void_p,
+                                        _i64, _c_void_p, _i32, _c_void_p, _i64, _i64,
+                                        _c_void_p, _c_void_p, _c_void_p, _sz, _c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
     "sfp8_layout_version": (_i32, []),
@@ -249,6 +253,55 @@ def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k,
                                             _stream(a_q.device))
     _check(st, "sfp8_sparse_linear_noalloc")
     return out
+
+
+def sfp8_sparse_linear_quant_workspace_bytes(m, n, k, device=None):
+    lib = load_library()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(lib.sfp8_sparse_linear_quant_workspace_bytes(m, n, k))
+
+
+def new_quant_workspace(m, n, k, device):
+    """A zeroed workspace for sfp8_sparse_linear_quant(m, n, k) on `device`."""
+    nbytes = sfp8_sparse_linear_quant_workspace_bytes(m, n, k, device)
+    return torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=device)
+
+
+def sfp8_sparse_linear_quant(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None, out=None,
+                             workspace=None, a_q=None, s_a=None):
+    """Quantise x [m, k] (bf16/f16/f32, unit column stride) row-wise and apply
+    the sparse linear, one library call: returns (y [m, n] bf16,
+    a_q [m, k] uint8, s_a [m] f32)."""
+    lib = load_library()
+    _require_cuda(x, packed, s_w, bias)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    m = x.shape[0]
+    if x.shape[1] != k:
+        raise ValueError("x has %d columns, expected k=%d" % (x.shape[1], k))
+    xd = TORCH_WIDE.get(x.dtype)
+    if xd is None:
+        raise ValueError("x dtype must be bfloat16, float16 or float32")
+    if bias is not None and bias.dtype != torch.bfloat16:
+        raise ValueError("bias must be bfloat16")
+    dev = x.device
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    if a_q is None:
+        a_q = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    if s_a is None:
+        s_a = torch.empty((m,), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = new_quant_workspace(m, n, k, dev)
+    ld = x.stride(0) if m > 1 else k
+    with torch.cuda.device(dev):
+        st = lib.sfp8_sparse_linear_quant(_ptr(x), DTYPE[xd], ld, DTYPE[_fp8_name(a_dtype)],
+                                          _ptr(a_q), _ptr(s_a), m, _ptr(packed),
+                                          DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n, k,
+                                          _ptr(bias), _ptr(out), _ptr(workspace),
+                                          workspace.numel(), _stream(dev))
+    _check(st, "sfp8_sparse_linear_quant")
+    return out, a_q, s_a
 
 
 def sfp8_read_device_status(clear=True):

@@ -767,6 +767,52 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype, const float*
                        partials, counters, static_cast<cudaStream_t>(stream));
 }
 
+size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % kStepK != 0) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  const LinearPlan pl = make_plan(m, n, k, sms);
+  return pl.partial_bytes + pl.counter_bytes;
+}
+
+sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
+                                     sfp8_dtype a_dtype, void* a_q, float* s_a, int64_t m,
+                                     const void* packed, sfp8_dtype w_dtype, const float* s_w,
+                                     int64_t n, int64_t k, const void* bias, void* y,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!is_wide(x_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (ld_x < k) return SFP8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK) return s;
+  if (m > 0 && x == nullptr) return SFP8_ERR_INVALID_ARG;
+  const int es = elem_size(x_dtype);
+  if (m > 0 && (!aligned(x, 16) || (ld_x * es) % 16 != 0)) return SFP8_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (empty) {
+    // n == 0 still quantises the activation; m == 0 does nothing
+    if (m == 0) return SFP8_OK;
+    return sfp8_quantize_rowwise(x, x_dtype, m, k, ld_x, a_q, a_dtype, s_a, stream);
+  }
+  const size_t need = pl.partial_bytes + pl.counter_bytes;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* partials = reinterpret_cast<float*>(ws);
+  unsigned int* counters = pl.counter_bytes > 0
+                               ? reinterpret_cast<unsigned int*>(ws + pl.partial_bytes)
+                               : nullptr;
+  s = sfp8_quantize_rowwise(x, x_dtype, m, k, ld_x, a_q, a_dtype, s_a, stream);
+  if (s != SFP8_OK) return s;
+  return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                       partials, counters, st);
+}
+
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
   if (flags == nullptr) return SFP8_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return SFP8_ERR_CUDA;

@@ -42,18 +42,23 @@ class SparseFp8Linear:
         return self
 
     def workspace(self, m):
+        """The layer's zeroed workspace for m tokens (kept between calls; each
+        call leaves its split-K counters at zero)."""
         ws = self._ws.get(m)
         if ws is None:
-            ws = B.new_workspace(m, self.n, self.k, self.device)
+            ws = B.new_quant_workspace(m, self.n, self.k, self.device)
             self._ws[m] = ws
         return ws
 
     def forward(self, x, out=None):
-        """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16."""
-        a_q, s_a = B.sfp8_quantize_rowwise(x, self.a_dtype)
-        return B.sfp8_sparse_linear(a_q, self.a_dtype, s_a, self.packed,
-                                    self.w_dtype, self.s_w, self.n, self.k, bias=self.bias,
-                                    out=out, workspace=self.workspace(x.shape[0]))
+        """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16.
+
+        One library call (sfp8_sparse_linear_quant): the quantiser, then the
+        GEMM as its programmatic dependent."""
+        y, _, _ = B.sfp8_sparse_linear_quant(x, self.a_dtype, self.packed, self.w_dtype,
+                                             self.s_w, self.n, self.k, bias=self.bias, out=out,
+                                             workspace=self.workspace(x.shape[0]))
+        return y
 
     __call__ = forward
 

@@ -115,3 +115,19 @@ def test_linear_validation_without_gpu(lib):
     assert na(FAKE, 0, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 4
     assert na(FAKE, 3, FAKE, 16, FAKE, 3, FAKE, 64, 0, None, FAKE, None) == 2
     assert na(FAKE, 3, FAKE, 0, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 0
+    fq = lib.sfp8_sparse_linear_quant
+    qargs = [FAKE, 0, 128, 3, FAKE, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE,
+             1 << 20, None]
+
+    def qcall(**kw):
+        a = list(qargs)
+        names = ["x", "x_dt", "ld_x", "a_dt", "a_q", "s_a", "m", "packed", "w_dt", "s_w",
+                 "n", "k", "bias", "y", "ws", "wsb", "stream"]
+        for key, v in kw.items():
+            a[names.index(key)] = v
+        return fq(*a)
+    assert qcall(x_dt=3) == 4          # x must be bf16 / f16 / f32
+    assert qcall(ld_x=64) == 1         # ld_x < k
+    assert qcall(a_dt=0) == 4          # a_q must be FP8
+    assert qcall(k=192, ld_x=192) == 2
+    assert qcall(m=0) == 0
