@@ -61,6 +61,34 @@ def test_exhaustive_bf16_sweep_scaled(fmt, amax):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_exhaustive_bf16_many_row_scales(fmt):
+    """Every finite bf16 value up to the row amax, for row amax values with
+    each of the 128 bf16 significands and exponents from 2^-60 to 2^60: the
+    quotients x / s fall on, next to and between FP8 rounding midpoints for
+    scales of every significand."""
+    rng = np.random.default_rng(7 if fmt == "e4m3" else 8)
+    sig = (np.arange(128, dtype=np.uint32) | 0x3F80).astype(np.uint32)          # [1, 2)
+    amax_bits = list(sig)
+    for e in range(-60, 61, 3):
+        amax_bits += list(((127 + e) << 7) | rng.integers(0, 128, size=2, dtype=np.uint32))
+    amaxes = (np.array(amax_bits, dtype=np.uint32) << 16).view(np.float32)
+    v_all = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32)
+    v_all = v_all[np.isfinite(v_all)]
+    width = 256
+    blocks = []
+    for a in amaxes:
+        v = v_all[np.abs(v_all) <= a]
+        v = np.concatenate([v, np.zeros((-v.size) % (width - 1), np.float32)])
+        body = v.reshape(-1, width - 1)
+        blocks.append(np.concatenate([np.full((body.shape[0], 1), a, np.float32), body], axis=1))
+    x = np.concatenate(blocks)
+    q, s = S.sfp8_quantize_rowwise(_to_dev(x, torch.bfloat16), fmt)
+    q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
 def _near_midpoint_rows(fmt, seed, n_rows):
     """fp32 rows whose quotients x / s fall within a few units in the last
     place of FP8 rounding midpoints (and on both sides of them)."""
@@ -92,9 +120,9 @@ def _near_midpoint_rows(fmt, seed, n_rows):
 
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
 def test_near_midpoint_quotients(fmt):
-    """The quantiser's division-free path must hand every quotient near an FP8
-    rounding midpoint to an exact division: codes equal the oracle's (IEEE
-    fp32 division, then one rounding) bit for bit."""
+    """The quantiser's division-free quotient must be exact next to every FP8
+    rounding midpoint: codes equal the oracle's (IEEE fp32 division, then one
+    rounding) bit for bit."""
     x = _near_midpoint_rows(fmt, 77 if fmt == "e4m3" else 78, 48)
     q, s = S.sfp8_quantize_rowwise(_to_dev(x, torch.float32), fmt)
     q_ref, s_ref = oracle.quantize_rowwise(x, fmt)
