@@ -145,6 +145,27 @@ sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n,
                              int64_t k, void* packed, void* stream);
 
 /*
+ * The whole weight preparation in one pass: sfp8_prune_24, then
+ * sfp8_quantize_rowwise (one scale per weight row n), then sfp8_compress_24,
+ * with the same results bit for bit (item 4's preparation of the weight at
+ * quantisation time, item 1's compressed format) but one read of w and no
+ * intermediate buffers.
+ *
+ *  w       device, [n, k] of w_dtype (BF16, F16 or F32), row stride ld_w >= k
+ *          elements; 16-byte aligned base, ld_w*size a 16-byte multiple.
+ *          Finite values (NaN/Inf are outside the contract).
+ *  q_dtype E4M3 or E5M2: the FP8 format of the compressed codes.
+ *  packed  device, sfp8_compressed_bytes(n, k) bytes, 16-byte aligned;
+ *          the layout of sfp8_compress_24.
+ *  s_w     device, [n] float32 (the row scales), 4-byte aligned.
+ *  k % 128 == 0, k > 0; n >= 0 (n == 0: nothing is launched).
+ * Validation errors return with nothing launched; buffers must not overlap.
+ */
+sfp8_status sfp8_prepare_weight_24(const void* w, sfp8_dtype w_dtype, int64_t n,
+                                   int64_t k, int64_t ld_w, sfp8_dtype q_dtype,
+                                   void* packed, float* s_w, void* stream);
+
+/*
  * Inverse of sfp8_compress_24 (a checking aid): writes the dense [n, k]
  * codes, 0x00 in dropped slots.  w_q 16-byte aligned, row stride k.
  * An invalid nibble sets SFP8_DEVICE_CHECK_FAIL in the device status word.

@@ -8,7 +8,7 @@ class on top of it, and the seeded synthetic-input generators.
 from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_quantize_rowwise, sfp8_prune_24, sfp8_padded_rows,
                       sfp8_compressed_bytes,
-                      sfp8_compress_24, sfp8_decompress_24,
+                      sfp8_compress_24, sfp8_decompress_24, sfp8_prepare_weight_24,
                       sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
                       sfp8_sparse_linear, sfp8_sparse_linear_noalloc,
                       sfp8_sparse_linear_quant, sfp8_sparse_linear_quant_workspace_bytes,
@@ -20,7 +20,7 @@ __all__ = [
     "Sfp8Error", "load_library", "library_path", "new_workspace",
     "sfp8_quantize_rowwise", "sfp8_prune_24", "sfp8_padded_rows",
     "sfp8_compressed_bytes",
-    "sfp8_compress_24", "sfp8_decompress_24",
+    "sfp8_compress_24", "sfp8_decompress_24", "sfp8_prepare_weight_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
     "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_sparse_linear_quant",
     "sfp8_sparse_linear_quant_workspace_bytes", "new_quant_workspace",

@@ -38,6 +38,8 @@ SIGNATURES = {
     "sfp8_compressed_bytes": (_sz, [_i64, _i64]),
     "sfp8_compress_24": (_i32, [_c_void_p, _i32, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_decompress_24": (_i32, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
+    "sfp8_prepare_weight_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _i32, _c_void_p,
+                                      _c_void_p, _c_void_p]),
     "sfp8_sparse_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "sfp8_workspace_clear": (_i32, [_c_void_p, _sz, _c_void_p]),
     "sfp8_sparse_linear": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _i32,
@@ -175,6 +177,31 @@ def sfp8_compress_24(w_q, w_dtype="e4m3", packed=None):
                                   _stream(w_q.device))
     _check(st, "sfp8_compress_24")
     return packed
+
+
+def sfp8_prepare_weight_24(w, q_dtype="e4m3", packed=None, scales=None):
+    """w [n, k] bf16/f16/f32 (unit column stride) -> (packed, s_w): prune 2:4,
+    quantise row-wise and compress in one pass (the same bytes as
+    sfp8_prune_24 -> sfp8_quantize_rowwise -> sfp8_compress_24)."""
+    lib = load_library()
+    _require_cuda(w)
+    if w.dim() != 2 or w.stride(1) != 1:
+        raise ValueError("w must be 2-D with unit column stride")
+    wd = TORCH_WIDE.get(w.dtype)
+    if wd is None:
+        raise ValueError("w dtype must be bfloat16, float16 or float32")
+    n, k = w.shape
+    if packed is None:
+        packed = torch.empty((lib.sfp8_compressed_bytes(n, k),), dtype=torch.uint8,
+                             device=w.device)
+    if scales is None:
+        scales = torch.empty((n,), dtype=torch.float32, device=w.device)
+    ld = w.stride(0) if n > 1 else k
+    with torch.cuda.device(w.device):
+        st = lib.sfp8_prepare_weight_24(_ptr(w), DTYPE[wd], n, k, ld, DTYPE[_fp8_name(q_dtype)],
+                                        _ptr(packed), _ptr(scales), _stream(w.device))
+    _check(st, "sfp8_prepare_weight_24")
+    return packed, scales
 
 
 def sfp8_decompress_24(packed, n, k, out=None):

@@ -13,6 +13,7 @@
 #include "device_common.cuh"
 #include "quantize_rowwise.cuh"
 #include "sparse24_pack.cuh"
+#include "prepare_weight24.cuh"
 #include "sparse_linear.cuh"
 #include "sparse_linear_pair.cuh"
 
@@ -704,10 +705,67 @@ sfp8_status sfp8_compress_24(const void* w_q, sfp8_dtype w_dtype, int64_t n, int
   DeviceInfo* dev = nullptr;
   sfp8_status s = current_device(&dev);
   if (s != SFP8_OK) return s;
-  dim3 grid(static_cast<unsigned>(k / kStepK), static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
+  dim3 grid(static_cast<unsigned>((k / kStepK + kCompressTiles - 1) / kCompressTiles),
+            static_cast<unsigned>(sfp8_padded_rows(n) / kTileN));
   compress24_kernel<<<grid, 512, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t*>(w_q), n, k, static_cast<uint8_t*>(packed));
   return launch_status();
+}
+
+extern "C++" {
+namespace {
+
+template <typename T>
+sfp8_status launch_prepare(const void* w, int64_t n, int64_t k, int64_t ld, sfp8_dtype q_dtype,
+                           void* packed, float* s_w, int sms, cudaStream_t st) {
+  const int64_t n_pad = sfp8_padded_rows(n);
+  auto kernel = q_dtype == SFP8_E4M3 ? prepare_weight24_kernel<T, SFP8_E4M3>
+                                     : prepare_weight24_kernel<T, SFP8_E5M2>;
+  // A grid-stride kernel: at most the co-resident blocks.  Rows longer than
+  // one register segment are re-read in sweep 2, so their rows in flight
+  // (one per warp) are also held to ~48 MB, well inside L2.
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, 32 * kPrepWarps, 0) !=
+          cudaSuccess || occ < 1)
+    occ = 1;
+  int64_t blocks = static_cast<int64_t>(occ) * sms;
+  const int64_t row_bytes = k * static_cast<int64_t>(sizeof(T));
+  if (row_bytes > 8192)
+    blocks = std::min<int64_t>(blocks, std::max<int64_t>(sms, (48ll << 20) / (row_bytes * kPrepWarps)));
+  blocks = std::min<int64_t>(blocks, n_pad / kPrepWarps);
+  kernel<<<static_cast<unsigned>(blocks), 32 * kPrepWarps, 0, st>>>(
+      static_cast<const T*>(w), n, k, ld, static_cast<uint8_t*>(packed), s_w, n_pad);
+  return launch_status();
+}
+
+}  // namespace
+}  // extern "C++"
+
+sfp8_status sfp8_prepare_weight_24(const void* w, sfp8_dtype w_dtype, int64_t n, int64_t k,
+                                   int64_t ld_w, sfp8_dtype q_dtype, void* packed, float* s_w,
+                                   void* stream) {
+  if (!is_fp8(q_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (w_dtype != SFP8_BF16 && w_dtype != SFP8_F16 && w_dtype != SFP8_F32)
+    return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (n < 0 || k < 0 || ld_w < k) return SFP8_ERR_INVALID_ARG;
+  if (k % kStepK != 0 || k == 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return SFP8_OK;
+  if (w == nullptr || packed == nullptr || s_w == nullptr) return SFP8_ERR_INVALID_ARG;
+  const int64_t esize = w_dtype == SFP8_F32 ? 4 : 2;
+  if (!aligned(w, 16) || (ld_w * esize) % 16 != 0 || !aligned(packed, 16) || !aligned(s_w, 4))
+    return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (w_dtype) {
+    case SFP8_BF16:
+      return launch_prepare<__nv_bfloat16>(w, n, k, ld_w, q_dtype, packed, s_w, dev->num_sms, st);
+    case SFP8_F16:
+      return launch_prepare<__half>(w, n, k, ld_w, q_dtype, packed, s_w, dev->num_sms, st);
+    default:
+      return launch_prepare<float>(w, n, k, ld_w, q_dtype, packed, s_w, dev->num_sms, st);
+  }
 }
 
 sfp8_status sfp8_decompress_24(const void* packed, int64_t n, int64_t k, void* w_q,

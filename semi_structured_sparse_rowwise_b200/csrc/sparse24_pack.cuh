@@ -91,49 +91,99 @@ __global__ void prune24_kernel(const Bits* __restrict__ w, int64_t rows, int64_t
 
 // ---------------------------------------------------------------- compress
 
-// Block = 512 threads = 128 rows x 4 threads; blockIdx.x = k tile, blockIdx.y
-// = row tile.  Each thread turns 32 input codes (8 groups) into 16 value
-// bytes and 4 metadata bytes.
+// The rank rule on a 4-code group, four bytes at a time.  With magnitudes
+// m_i = code_i & 0x7F (7 bits), the byte (0x80 | m_x) - m_y needs no borrow and
+// has its top bit set iff m_x >= m_y.  Two such subtractions per pair of groups
+// give the six comparisons of each group (i beats j for i < j iff m_i >= m_j),
+// and a 64-entry table indexed by those six bits gives the byte selector of the
+// two kept codes and their index nibble.
+//
+// Table index bits: 0: m0>=m1, 1: m0>=m2, 2: m0>=m3, 3: m1>=m2, 4: m1>=m3, 5: m2>=m3.
+// Entry for the first group of a pair:  byte selector i0 | i1 << 4 in bits 0..7,
+//   nibble in bits 16..19.
+// Entry for the second group: byte selector (4 + i0) | (4 + i1) << 4 in bits 8..15,
+//   nibble in bits 20..23.
+__device__ __forceinline__ void group_select_entries(uint32_t idx, uint32_t& first,
+                                                     uint32_t& second) {
+  const uint32_t b01 = idx & 1, b02 = (idx >> 1) & 1, b03 = (idx >> 2) & 1;
+  const uint32_t b12 = (idx >> 3) & 1, b13 = (idx >> 4) & 1, b23 = (idx >> 5) & 1;
+  const uint32_t beaten0 = (1 - b01) + (1 - b02) + (1 - b03);
+  const uint32_t beaten1 = b01 + (1 - b12) + (1 - b13);
+  const uint32_t beaten2 = b02 + b12 + (1 - b23);
+  const uint32_t beaten3 = b03 + b13 + b23;
+  const uint32_t keep = (beaten0 < 2 ? 1u : 0u) | (beaten1 < 2 ? 2u : 0u) |
+                        (beaten2 < 2 ? 4u : 0u) | (beaten3 < 2 ? 8u : 0u);
+  uint32_t i0 = 0, i1 = 1;
+  if (__popc(keep) == 2) kept_indices(keep, i0, i1);   // always, for real comparisons
+  const uint32_t nib = i0 | (i1 << 2);
+  first = i0 | (i1 << 4) | (nib << 16);
+  second = ((4 + i0) << 8) | ((4 + i1) << 12) | (nib << 20);
+}
+
+// Top bits of the four bytes of d, gathered into bits 28..31 (byte 0's in bit
+// 28).  The partial products land on distinct bit positions, so nothing carries.
+__device__ __forceinline__ uint32_t byte_signs_high(uint32_t d) {
+  return (d & 0x80808080u) * 0x00204081u;
+}
+
+// Block = 512 threads = 128 rows x 4 threads; blockIdx.x covers kCompressTiles
+// k tiles, blockIdx.y = row tile.  For each of its k tiles a thread turns 32
+// input codes (8 groups) into 16 value bytes and 4 metadata bytes; all its
+// loads are issued before the first group is selected.
+constexpr int kCompressTiles = 2;
+
 __global__ void __launch_bounds__(512)
     compress24_kernel(const uint8_t* __restrict__ wq, int64_t n, int64_t k,
                       uint8_t* __restrict__ packed) {
+  __shared__ uint32_t tab_first[64], tab_second[64];
+  if (threadIdx.x < 64) group_select_entries(threadIdx.x, tab_first[threadIdx.x],
+                                             tab_second[threadIdx.x]);
+  __syncthreads();
   const int r = threadIdx.x / 4;   // row inside the tile
   const int j = threadIdx.x % 4;   // 32-code chunk inside the 128-wide k tile
-  const int64_t kt = blockIdx.x;
   const int64_t nt = blockIdx.y;
   const int64_t row = nt * 128 + r;
   const int64_t ktiles = k / 128;
-  uint32_t vout[4];
-  uint32_t mout = 0;
-  if (row < n) {
-    const uint8_t* src = wq + row * k + kt * 128 + 32 * j;
-    uint32_t in[8];
-    *reinterpret_cast<uint4*>(&in[0]) = __ldg(reinterpret_cast<const uint4*>(src));
-    *reinterpret_cast<uint4*>(&in[4]) = __ldg(reinterpret_cast<const uint4*>(src + 16));
-    uint32_t vb[16];
+  const int64_t kt0 = static_cast<int64_t>(blockIdx.x) * kCompressTiles;
+  uint32_t in[kCompressTiles][8];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      const uint32_t word = in[g];   // codes 4g..4g+3 of this chunk, little-endian
-      const uint32_t c0 = word & 0xFF, c1 = (word >> 8) & 0xFF, c2 = (word >> 16) & 0xFF,
-                     c3 = word >> 24;
-      const uint32_t keep = keep_mask4(c0 & 0x7F, c1 & 0x7F, c2 & 0x7F, c3 & 0x7F);
-      uint32_t i0, i1;
-      kept_indices(keep, i0, i1);
-      vb[2 * g] = (word >> (8 * i0)) & 0xFF;
-      vb[2 * g + 1] = (word >> (8 * i1)) & 0xFF;
-      mout |= (i0 | (i1 << 2)) << (4 * g);
+  for (int t = 0; t < kCompressTiles; ++t) {
+    if (row < n && kt0 + t < ktiles) {
+      const uint8_t* src = wq + row * k + (kt0 + t) * 128 + 32 * j;
+      *reinterpret_cast<uint4*>(&in[t][0]) = __ldg(reinterpret_cast<const uint4*>(src));
+      *reinterpret_cast<uint4*>(&in[t][4]) = __ldg(reinterpret_cast<const uint4*>(src + 16));
+    } else {
+#pragma unroll
+      for (int g = 0; g < 8; ++g) in[t][g] = 0;   // all-zero groups select (0, 1): nibble 0x4
     }
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-      vout[w] = vb[4 * w] | (vb[4 * w + 1] << 8) | (vb[4 * w + 2] << 16) | (vb[4 * w + 3] << 24);
-  } else {
-    vout[0] = vout[1] = vout[2] = vout[3] = 0;
-    mout = 0x44444444u;   // indices (0, 1) in every group
   }
-  uint8_t* tile = packed + (nt * ktiles + kt) * 10240;
-  *reinterpret_cast<uint4*>(tile + 64 * r + 16 * (j ^ ((r >> 1) & 3))) =
-      make_uint4(vout[0], vout[1], vout[2], vout[3]);
-  *reinterpret_cast<uint32_t*>(tile + 8192 + 16 * r + 4 * j) = mout;
+#pragma unroll
+  for (int t = 0; t < kCompressTiles; ++t) {
+    if (kt0 + t >= ktiles) break;
+    uint32_t vout[4];
+    uint32_t mout = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const uint32_t wa = in[t][2 * p], wb = in[t][2 * p + 1];
+      const uint32_t la = wa & 0x7F7F7F7Fu, lb = wb & 0x7F7F7F7Fu;
+      const uint32_t ha = wa | 0x80808080u, hb = wb | 0x80808080u;
+      // bytes (m0>=m1, m0>=m2, m0>=m3, m1>=m2) of each group
+      const uint32_t da = __byte_perm(ha, 0, 0x1000) - __byte_perm(la, 0, 0x2321);
+      const uint32_t db = __byte_perm(hb, 0, 0x1000) - __byte_perm(lb, 0, 0x2321);
+      // bytes (a: m1>=m3, m2>=m3; b: m1>=m3, m2>=m3)
+      const uint32_t d2 = __byte_perm(ha, hb, 0x6521) - __byte_perm(la, lb, 0x7733);
+      const uint32_t s2 = byte_signs_high(d2) >> 24;   // bits 4..7
+      const uint32_t ia = (byte_signs_high(da) >> 28) | (s2 & 0x30u);
+      const uint32_t ib = (byte_signs_high(db) >> 28) | ((s2 >> 2) & 0x30u);
+      const uint32_t e = tab_first[ia] | tab_second[ib];
+      vout[p] = __byte_perm(wa, wb, e & 0xFFFFu);
+      mout |= (e >> 16) << (8 * p);
+    }
+    uint8_t* tile = packed + (nt * ktiles + kt0 + t) * 10240;
+    *reinterpret_cast<uint4*>(tile + 64 * r + 16 * (j ^ ((r >> 1) & 3))) =
+        make_uint4(vout[0], vout[1], vout[2], vout[3]);
+    *reinterpret_cast<uint32_t*>(tile + 8192 + 16 * r + 4 * j) = mout;
+  }
 }
 
 // Inverse: same thread mapping, n real rows only.

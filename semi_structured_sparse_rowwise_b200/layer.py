@@ -23,9 +23,12 @@ class SparseFp8Linear:
         self.w_dtype = w_dtype
         self.a_dtype = a_dtype
         self.device = weight.device
-        w = B.sfp8_prune_24(weight.contiguous()) if prune else weight.contiguous()
-        w_q, self.s_w = B.sfp8_quantize_rowwise(w, w_dtype)
-        self.packed = B.sfp8_compress_24(w_q, w_dtype)
+        if prune:
+            # prune, quantise and compress in one pass over the weight
+            self.packed, self.s_w = B.sfp8_prepare_weight_24(weight.contiguous(), w_dtype)
+        else:
+            w_q, self.s_w = B.sfp8_quantize_rowwise(weight.contiguous(), w_dtype)
+            self.packed = B.sfp8_compress_24(w_q, w_dtype)
         self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
         self._ws = {}
 

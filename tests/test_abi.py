@@ -87,6 +87,20 @@ def test_prune_compress_validation_without_gpu(lib):
     assert lib.sfp8_decompress_24(FAKE, 4, 100, FAKE, None) == 2
 
 
+def test_prepare_weight_validation_without_gpu(lib):
+    f = lib.sfp8_prepare_weight_24
+    assert f(FAKE, 0, 4, 128, 128, 0, FAKE, FAKE, None) == 4        # codes must be FP8
+    assert f(FAKE, 3, 4, 128, 128, 3, FAKE, FAKE, None) == 4        # input must be wide
+    assert f(FAKE, 0, 4, 192, 192, 3, FAKE, FAKE, None) == 2        # k % 128
+    assert f(FAKE, 0, 4, 0, 0, 3, FAKE, FAKE, None) == 2
+    assert f(FAKE, 0, 4, 128, 64, 3, FAKE, FAKE, None) == 1         # ld < k
+    assert f(FAKE, 0, 0, 128, 128, 3, FAKE, FAKE, None) == 0        # nothing to do
+    assert f(FAKE, 0, 4, 128, 128, 3, FAKE, None, None) == 1        # no scales
+    assert f(FAKE_ODD, 0, 4, 128, 128, 3, FAKE, FAKE, None) == 3
+    assert f(FAKE, 0, 4, 128, 132, 3, FAKE, FAKE, None) == 3        # row stride 264 bytes
+    assert f(FAKE, 0, 4, 128, 128, 3, FAKE_ODD, FAKE, None) == 3
+
+
 def test_linear_validation_without_gpu(lib):
     f = lib.sfp8_sparse_linear
     args = [FAKE, 3, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE, 1 << 20, None]
