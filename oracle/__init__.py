@@ -21,6 +21,9 @@ OCP 8-bit floating point specification (OFP8), which defines e4m3 and e5m2:
 * :mod:`oracle.fp8`       FP8 decode tables from the bit fields; RNE+satfinite
                           encoder.
 * :mod:`oracle.quantize`  per-row amax, scale, divide, encode.
+* :mod:`oracle.quantize_tensor`  the same with one amax for the whole tensor
+                          (page "[float8nocompile] ...", pytorch/ao pull
+                          request 1455).
 * :mod:`oracle.prune`     2:4 magnitude prune of a 16/32-bit weight.
 * :mod:`oracle.compress`  2:4 compression to kept codes + index nibbles, and
                           its inverse.
@@ -37,6 +40,7 @@ from .fp8 import (E4M3, E5M2, FORMATS, decode_table, decode, fp8_max,
                   max_code, encode_rne_sat, bf16_bits_to_f32, f16_bits_to_f32,
                   round_to_bf16)
 from .quantize import quantize_rowwise, GUARD_AMAX
+from .quantize_tensor import quantize_tensorwise
 from .prune import prune_24
 from .compress import compress_24, decompress_24, NIBBLES_VALID
 from .layout import unpack_physical, padded_rows, packed_bytes
@@ -45,7 +49,7 @@ from .linear import sparse_linear_ref, acceptance_bound, check_linear
 __all__ = [
     "E4M3", "E5M2", "FORMATS", "decode_table", "decode", "fp8_max", "max_code",
     "encode_rne_sat", "bf16_bits_to_f32", "f16_bits_to_f32", "round_to_bf16",
-    "quantize_rowwise", "GUARD_AMAX", "prune_24", "compress_24",
+    "quantize_rowwise", "quantize_tensorwise", "GUARD_AMAX", "prune_24", "compress_24",
     "decompress_24", "NIBBLES_VALID", "unpack_physical", "padded_rows",
     "packed_bytes", "sparse_linear_ref", "acceptance_bound",
     "check_linear",

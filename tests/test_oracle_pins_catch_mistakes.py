@@ -141,3 +141,28 @@ def test_prune_mistakes_are_caught(monkeypatch):
     monkeypatch.setattr(prune_mod, "prune_24", lambda w: np.where(
         real(np.abs(w.reshape(-1, 1, 4)).astype(np.float64)).reshape(w.shape) < 2, w, np.float32(-0.0)))
     assert not _prune_pin(prune_mod.prune_24)
+
+
+def _global_amax_pin(quantize_tensorwise):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((6, 40)).astype(np.float32)
+    x *= np.float32(2.0) ** np.arange(6, dtype=np.float32)[:, None]
+    q, s = quantize_tensorwise(x, E4M3)
+    return (np.size(s) == 1 and np.float32(s) == np.float32(np.max(np.abs(x)) / np.float32(448.0))
+            and np.array_equal(q, oracle.quantize_rowwise(x.reshape(1, -1), E4M3)[0].reshape(x.shape)))
+
+
+def test_tensorwise_mistakes_are_caught():
+    def per_block_amax(x, fmt):          # each block (row) scaled by its own amax
+        q, s = oracle.quantize_rowwise(np.asarray(x, np.float32), fmt)
+        return q, s
+
+    def last_block_amax(x, fmt):         # a race: the amax read before the last block folded in
+        x = np.asarray(x, np.float32)
+        amax = np.float32(np.max(np.abs(x[:-1])))
+        s = np.float32(amax / np.float32(oracle.fp8_max(fmt)))
+        return oracle.encode_rne_sat((x / s).astype(np.float32), fmt), s
+
+    assert _global_amax_pin(oracle.quantize_tensorwise)
+    assert not _global_amax_pin(per_block_amax)
+    assert not _global_amax_pin(last_block_amax)
