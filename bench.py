@@ -526,14 +526,99 @@ def run_ours(args):
     return 0
 
 
+# ----------------------------------------------------------------- tensor-wise quantiser
+
+# The conversion sizes of the page "[float8nocompile] Add alternate Triton
+# kernels for FP8 conversion ..." (pytorch/ao pull request 1455), its tables.
+TENSORWISE_SIZES = (65500, 1 << 20, 1 << 24, 1 << 28)
+
+
+def run_tensorwise(args):
+    """Times sfp8_quantize_tensorwise (both amax modes, bf16 and fp32 input,
+    e4m3 output) on the pages' conversion sizes.  Each timed call follows a
+    256 MB write that evicts the input from L2; CUDA events bracket the call
+    alone, and the median over the repetitions is reported (`us`); `us_warm`
+    is the mean of back-to-back calls without the flush."""
+    import torch
+    rank, local, world = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import semi_structured_sparse_rowwise_b200 as S
+    S.load_library()
+    peak, peak_kind = measured_peaks()
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev).manual_seed(1004)
+    reps = max(args.steps, 5)
+    table = []
+    with ClockSampler(local) as clk:
+        for dtype in (torch.float32, torch.bfloat16):
+            for numel in TENSORWISE_SIZES:
+                x = torch.randn(numel, generator=g, device=dev, dtype=torch.float32).to(dtype)
+                q = torch.empty((numel,), dtype=torch.uint8, device=dev)
+                sc = torch.empty((1,), dtype=torch.float32, device=dev)
+                for mode in ("reduce", "atomic"):
+                    ws = S.new_tensorwise_workspace(mode, dev)
+                    for _ in range(args.warmup):
+                        S.sfp8_quantize_tensorwise(x, "e4m3", mode, q=q, scale=sc, workspace=ws)
+                    ev = [(torch.cuda.Event(enable_timing=True),
+                           torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+                    torch.cuda.synchronize(dev)
+                    for e0, e1 in ev:
+                        flush.fill_(1)
+                        e0.record()
+                        S.sfp8_quantize_tensorwise(x, "e4m3", mode, q=q, scale=sc, workspace=ws)
+                        e1.record()
+                    torch.cuda.synchronize(dev)
+                    times = sorted(e0.elapsed_time(e1) * 1e3 for e0, e1 in ev)
+                    us = times[len(times) // 2]
+                    # warm: back-to-back calls, no flush (the input stays in
+                    # L2 when it fits), the mean over the repetitions
+                    w0, w1 = (torch.cuda.Event(enable_timing=True),
+                              torch.cuda.Event(enable_timing=True))
+                    w0.record()
+                    for _ in range(reps):
+                        S.sfp8_quantize_tensorwise(x, "e4m3", mode, q=q, scale=sc, workspace=ws)
+                    w1.record()
+                    w1.synchronize()
+                    us_warm = w0.elapsed_time(w1) * 1e3 / reps
+                    alg = numel * (x.element_size() + 1) + 4
+                    table.append({"numel": numel, "dtype": str(dtype).replace("torch.", ""),
+                                  "mode": mode, "us": us, "GB/s": alg / (us * 1e-6) / 1e9,
+                                  "frac": alg / (us * 1e-6) / 1e9 / peak, "us_warm": us_warm})
+                del x, q
+    st, flags = S.sfp8_read_device_status(clear=True)
+    if st != 0:
+        raise RuntimeError("device status %d flags %#x" % (st, flags))
+    big = [r for r in table if r["numel"] == TENSORWISE_SIZES[-1]]
+    best = max(big, key=lambda r: r["GB/s"])
+    line = {
+        "metric": "tensor-wise FP8 quantise GB/s (one global amax)", "value": best["GB/s"],
+        "unit": "GB/s", "n_gpus": world, "steps": reps, "warmup": args.warmup,
+        "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": "quantize_tensorwise", "sizes": list(TENSORWISE_SIZES),
+                   "l2": "256 MB write before every timed call", "seed": 1004},
+        "roofline": {"bound": "hbm", "achieved": best["GB/s"], "peak": peak, "unit": "GB/s",
+                     "frac": best["GB/s"] / peak, "traffic": None,
+                     "kernel": "quantize_tensorwise_kernel",
+                     "algorithmic_bytes": "numel * (input bytes + 1) + 4 (one read, one write)",
+                     "peak_source": peak_kind},
+        "table": table, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--m", type=int, default=16, choices=[1, 4, 16])
-    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "prefill_8b"],
-                    help="decode gate/up (default, GB/s) or the prefill linears (TFLOP/s)")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[WORKLOAD, "prefill_8b", "quantize_tensorwise"],
+                    help="decode gate/up (default, GB/s), the prefill linears (TFLOP/s), or "
+                    "the standalone tensor-wise quantiser on the pages' conversion sizes")
     ap.add_argument("--shape", type=int, default=2, choices=[0, 1, 2, 3],
                     help="prefill_8b shape: 0 QKV, 1 O, 2 up (default), 3 down")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -545,6 +630,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "quantize_tensorwise":
+        return run_tensorwise(args)
     return run_ours(args)
 
 

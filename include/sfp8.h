@@ -94,6 +94,54 @@ sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype,
                                   void* stream);
 
 /*
+ * How sfp8_quantize_tensorwise finds the global amax (page "[float8nocompile]
+ * Add alternate Triton kernels for FP8 conversion which use atomic_max-based
+ * algo instead of reduction-based algo", pytorch/ao pull request 1455,
+ * Summary and review): REDUCE writes one partial maximum per block and
+ * reduces them; ATOMIC folds every block's maximum into one word with an
+ * atomic max, so it needs no buffer sized by the block count.  A maximum is
+ * exact in any order: both modes give the same bits.
+ */
+typedef enum {
+  SFP8_AMAX_REDUCE = 0,
+  SFP8_AMAX_ATOMIC = 1
+} sfp8_amax_mode;
+
+/*
+ * Workspace bytes of sfp8_quantize_tensorwise on the current device:
+ * 64 for ATOMIC, 64 + 16 * (number of SMs) for REDUCE; 0 for an unknown mode.
+ */
+size_t sfp8_quantize_tensorwise_workspace_bytes(sfp8_amax_mode mode);
+
+/*
+ * Tensor-wise (one scale) FP8 quantisation of a contiguous tensor of numel
+ * elements -- the row-wise rule above with the whole tensor as the one row:
+ *     amax  = max_i |x[i]|                        (fp32, exact)
+ *     s     = max(amax, 1e-12f) / FP8_MAX          (IEEE fp32 division)
+ *     q[i]  = RNE_satfinite_fp8(x[i] / s)          (IEEE fp32 division,
+ *                                                   then one rounding)
+ * One launch (a cooperative grid: both sweeps over x, the amax between them
+ * through a grid barrier in the workspace).
+ *
+ *  x       device, numel elements of x_dtype (BF16, F16 or F32), contiguous,
+ *          16-byte aligned.  Any numel >= 0 (numel == 0 writes the guard
+ *          scale 1e-12f / FP8_MAX).
+ *  q       device, numel bytes (q_dtype E4M3 or E5M2), 16-byte aligned.
+ *  scale   device, one float32 (s above), written.
+ *  workspace  device, >= sfp8_quantize_tensorwise_workspace_bytes(mode)
+ *          bytes, 16-byte aligned, zero before its first use (e.g. by
+ *          sfp8_workspace_clear); every call leaves it ready for the next.
+ *          Calls that share a workspace must not overlap on the GPU; clear
+ *          it again after a call that reported a device error.
+ * A barrier wait that runs out its time limit sets SFP8_DEVICE_TIMEOUT and
+ * leaves q unwritten.
+ */
+sfp8_status sfp8_quantize_tensorwise(const void* x, sfp8_dtype x_dtype, int64_t numel,
+                                     void* q, sfp8_dtype q_dtype, float* scale,
+                                     sfp8_amax_mode mode, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
  * 2:4 magnitude pruning along the row (the weight preparation that the
  * page's "sparsify/quantize method" performs before quantisation): in every
  * group of four consecutive elements keep the two of largest |w| (-0.0 is
@@ -215,6 +263,84 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype,
                                const float* s_w, int64_t n, int64_t k,
                                const void* bias, void* y, void* workspace,
                                size_t workspace_bytes, void* stream);
+
+/*
+ * Work-split selection ("algorithms") of the sparse linear.  The page "Add
+ * CUTLASS-based row-wise scaled sparse FP8 kernel" (pytorch/ao pull request
+ * 1671) leaves "a meaningful config selection" as future work, and the page
+ * "Add algorithm search to FP8 sparse linear benchmark" (pytorch/ao #4432)
+ * threads an algorithm id through the sparse matmul and finds the fastest
+ * one per shape with a search call.  Here an algorithm is one work split of
+ * the GEMM for a shape (m, n, k): the kernel (one CTA per tile, or CTA pairs
+ * sharing a 256-row tile), the token-tile width, the k steps per pipeline
+ * stage, the weight tiles per CTA and the whole-tile / stream-K split.
+ * Algorithm 0 is the built-in rule; the list depends on the shape and the
+ * device's SM count.  Every algorithm computes the same y up to the fp32
+ * summation order (within the tolerance of sfp8_sparse_linear; each one is
+ * deterministic).
+ */
+
+/* Number of algorithms for (m, n, k) on the current device (0 for an
+ * unsupported shape). */
+int sfp8_sparse_linear_algo_count(int64_t m, int64_t n, int64_t k);
+
+/* Description of one algorithm: info[0..7] = {pair kernel (0/1), tokens per
+ * tile, k steps per stage, weight tiles per CTA, whole tiles (1) or
+ * stream-K (0), activation resident in shared memory (0/1), pipeline stages,
+ * CTAs launched (pairs: at most; the count is capped at launch by the
+ * co-resident clusters)}. */
+sfp8_status sfp8_sparse_linear_algo_info(int64_t m, int64_t n, int64_t k, int algo,
+                                         int32_t* info);
+
+/* Workspace bytes of one algorithm, and the most over all algorithms of the
+ * shape (what sfp8_sparse_linear_search needs). */
+size_t sfp8_sparse_linear_algo_workspace_bytes(int64_t m, int64_t n, int64_t k, int algo);
+size_t sfp8_sparse_linear_search_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/* sfp8_sparse_linear with an explicit algorithm (0 <= algo < count, else
+ * SFP8_ERR_INVALID_ARG); arguments otherwise as sfp8_sparse_linear, the
+ * workspace sized by sfp8_sparse_linear_algo_workspace_bytes. */
+sfp8_status sfp8_sparse_linear_algo(const void* a_q, sfp8_dtype a_dtype,
+                                    const float* s_a, int64_t m,
+                                    const void* packed, sfp8_dtype w_dtype,
+                                    const float* s_w, int64_t n, int64_t k,
+                                    const void* bias, void* y, int algo,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/*
+ * Times every algorithm of the shape on the caller's buffers and returns the
+ * fastest in *best_algo (times_us[i], when given, receives algorithm i's
+ * median time in microseconds for i < times_len).  Each algorithm runs once
+ * untimed, then `reps` (1..64) times, each launch bracketed by CUDA events on
+ * `stream`; when `flush` is given, flush_bytes of it are overwritten before
+ * every timed launch (a buffer larger than L2 makes each launch read its
+ * operands from HBM).  Synchronous: it waits for the stream.  y and the
+ * workspace (>= sfp8_sparse_linear_search_workspace_bytes) are overwritten,
+ * and the workspace is left zeroed only in the parts the last algorithm
+ * used -- clear it before giving it to sfp8_sparse_linear.  Not for use
+ * inside a stream capture.
+ */
+sfp8_status sfp8_sparse_linear_search(const void* a_q, sfp8_dtype a_dtype,
+                                      const float* s_a, int64_t m,
+                                      const void* packed, sfp8_dtype w_dtype,
+                                      const float* s_w, int64_t n, int64_t k,
+                                      const void* bias, void* y, void* workspace,
+                                      size_t workspace_bytes, void* flush,
+                                      size_t flush_bytes, int reps, int* best_algo,
+                                      float* times_us, int times_len, void* stream);
+
+/*
+ * The shape-keyed table of the current device: after
+ * sfp8_sparse_linear_set_algo(m, n, k, a) with a > 0, sfp8_sparse_linear,
+ * sfp8_sparse_linear_quant, sfp8_sparse_linear_noalloc and their workspace
+ * queries use algorithm a for exactly that (m, n, k); a <= 0 removes the
+ * entry (back to the built-in rule).  Query workspace sizes after setting.
+ * Thread-safe; the table lives until the process exits.
+ * sfp8_sparse_linear_get_algo returns the entry (0 when none).
+ */
+sfp8_status sfp8_sparse_linear_set_algo(int64_t m, int64_t n, int64_t k, int algo);
+int sfp8_sparse_linear_get_algo(int64_t m, int64_t n, int64_t k);
 
 /*
  * Workspace for sfp8_sparse_linear_quant (the same as sfp8_sparse_linear's

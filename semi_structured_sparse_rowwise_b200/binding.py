@@ -25,6 +25,7 @@ STATUS_NAMES = {
 }
 DTYPE = {"bf16": 0, "f16": 1, "f32": 2, "e4m3": 3, "e5m2": 4}
 TORCH_WIDE = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}
+AMAX_MODE = {"reduce": 0, "atomic": 1}
 DEVICE_TIMEOUT = 0x1
 DEVICE_CHECK_FAIL = 0x2
 
@@ -33,6 +34,9 @@ _c_void_p, _i64, _sz, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, c
 SIGNATURES = {
     "sfp8_quantize_rowwise": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _i32,
                                      _c_void_p, _c_void_p]),
+    "sfp8_quantize_tensorwise_workspace_bytes": (_sz, [_i32]),
+    "sfp8_quantize_tensorwise": (_i32, [_c_void_p, _i32, _i64, _c_void_p, _i32, _c_void_p, _i32,
+                                        _c_void_p, _sz, _c_void_p]),
     "sfp8_prune_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_padded_rows": (_i64, [_i64]),
     "sfp8_compressed_bytes": (_sz, [_i64, _i64]),
@@ -48,6 +52,21 @@ SIGNATURES = {
     "sfp8_sparse_linear_noalloc": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p,
                                           _i32, _c_void_p, _i64, _i64, _c_void_p,
                                           _c_void_p, _c_void_p]),
+    "sfp8_sparse_linear_algo_count": (_i32, [_i64, _i64, _i64]),
+    "sfp8_sparse_linear_algo_info": (_i32, [_i64, _i64, _i64, _i32,
+                                            ctypes.POINTER(ctypes.c_int32)]),
+    "sfp8_sparse_linear_algo_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32]),
+    "sfp8_sparse_linear_search_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "sfp8_sparse_linear_algo": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _i32,
+                                       _c_void_p, _i64, _i64, _c_void_p, _c_void_p, _i32,
+                                       _c_void_p, _sz, _c_void_p]),
+    "sfp8_sparse_linear_search": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _i32,
+                                         _c_void_p, _i64, _i64, _c_void_p, _c_void_p,
+                                         _c_void_p, _sz, _c_void_p, _sz, _i32,
+                                         ctypes.POINTER(ctypes.c_int32),
+                                         ctypes.POINTER(ctypes.c_float), _i32, _c_void_p]),
+    "sfp8_sparse_linear_set_algo": (_i32, [_i64, _i64, _i64, _i32]),
+    "sfp8_sparse_linear_get_algo": (_i32, [_i64, _i64, _i64]),
     "sfp8_sparse_linear_quant_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "sfp8_sparse_linear_quant": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p, _c_void_p,
                                         _i64, _c_void_p, _i32, _c_void_p, _i64, _i64,
@@ -133,6 +152,47 @@ def sfp8_quantize_rowwise(x, q_dtype="e4m3", q=None, scales=None):
                                        DTYPE[_fp8_name(q_dtype)], _ptr(scales), _stream(x.device))
     _check(st, "sfp8_quantize_rowwise")
     return q, scales
+
+
+def sfp8_quantize_tensorwise_workspace_bytes(mode="reduce", device=None):
+    lib = load_library()
+    with torch.cuda.device(device if device is not None else torch.cuda.current_device()):
+        return int(lib.sfp8_quantize_tensorwise_workspace_bytes(AMAX_MODE[mode]))
+
+
+def new_tensorwise_workspace(mode, device):
+    """A zeroed workspace for sfp8_quantize_tensorwise on `device`."""
+    nbytes = sfp8_quantize_tensorwise_workspace_bytes(mode, device)
+    return torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=device)
+
+
+def sfp8_quantize_tensorwise(x, q_dtype="e4m3", mode="reduce", q=None, scale=None,
+                             workspace=None):
+    """x (any shape, contiguous) bf16/f16/f32 -> (q uint8 of x's shape, scale f32 [1]):
+    one scale for the whole tensor, the global amax found by `mode`
+    ('reduce': per-block partials, 'atomic': one word with atomic max)."""
+    lib = load_library()
+    _require_cuda(x)
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    xd = TORCH_WIDE.get(x.dtype)
+    if xd is None:
+        raise ValueError("x dtype must be bfloat16, float16 or float32")
+    if mode not in AMAX_MODE:
+        raise ValueError("mode must be 'reduce' or 'atomic'")
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = new_tensorwise_workspace(mode, x.device)
+    with torch.cuda.device(x.device):
+        st = lib.sfp8_quantize_tensorwise(_ptr(x), DTYPE[xd], x.numel(), _ptr(q),
+                                          DTYPE[_fp8_name(q_dtype)], _ptr(scale),
+                                          AMAX_MODE[mode], _ptr(workspace), workspace.numel(),
+                                          _stream(x.device))
+    _check(st, "sfp8_quantize_tensorwise")
+    return q, scale
 
 
 def sfp8_prune_24(w, out=None):
@@ -280,6 +340,95 @@ def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k,
                                             _stream(a_q.device))
     _check(st, "sfp8_sparse_linear_noalloc")
     return out
+
+
+ALGO_FIELDS = ("pair", "bn", "ks", "wt", "whole_tiles", "ra", "stages", "grid")
+
+
+def _dev_ctx(device):
+    return torch.cuda.device(device if device is not None else torch.cuda.current_device())
+
+
+def sfp8_sparse_linear_algo_count(m, n, k, device=None):
+    with _dev_ctx(device):
+        return int(load_library().sfp8_sparse_linear_algo_count(m, n, k))
+
+
+def sfp8_sparse_linear_algo_info(m, n, k, algo, device=None):
+    """dict of the algorithm's work split (keys ALGO_FIELDS)."""
+    info = (ctypes.c_int32 * 8)()
+    with _dev_ctx(device):
+        st = load_library().sfp8_sparse_linear_algo_info(m, n, k, algo, info)
+    _check(st, "sfp8_sparse_linear_algo_info")
+    return dict(zip(ALGO_FIELDS, [int(v) for v in info]))
+
+
+def sfp8_sparse_linear_algo_workspace_bytes(m, n, k, algo, device=None):
+    with _dev_ctx(device):
+        return int(load_library().sfp8_sparse_linear_algo_workspace_bytes(m, n, k, algo))
+
+
+def sfp8_sparse_linear_search_workspace_bytes(m, n, k, device=None):
+    with _dev_ctx(device):
+        return int(load_library().sfp8_sparse_linear_search_workspace_bytes(m, n, k))
+
+
+def sfp8_sparse_linear_algo(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, algo, bias=None,
+                            out=None, workspace=None):
+    """sfp8_sparse_linear with an explicit work split (algorithm index)."""
+    lib = load_library()
+    _require_cuda(a_q, s_a, packed, s_w, bias)
+    if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
+        raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
+    m = a_q.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
+    if workspace is None:
+        nbytes = sfp8_sparse_linear_algo_workspace_bytes(m, n, k, algo, a_q.device)
+        workspace = torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=a_q.device)
+    with torch.cuda.device(a_q.device):
+        st = lib.sfp8_sparse_linear_algo(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
+                                         _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n,
+                                         k, _ptr(bias), _ptr(out), algo, _ptr(workspace),
+                                         workspace.numel(), _stream(a_q.device))
+    _check(st, "sfp8_sparse_linear_algo")
+    return out
+
+
+def sfp8_sparse_linear_search(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bias=None,
+                              reps=10, flush=None, out=None):
+    """Times every work split of the shape (see include/sfp8.h); returns
+    (best algorithm, [median microseconds per algorithm])."""
+    lib = load_library()
+    _require_cuda(a_q, s_a, packed, s_w, bias, flush)
+    m = a_q.shape[0]
+    dev = a_q.device
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    count = sfp8_sparse_linear_algo_count(m, n, k, dev)
+    nbytes = sfp8_sparse_linear_search_workspace_bytes(m, n, k, dev)
+    ws = torch.zeros((max(nbytes, 16),), dtype=torch.uint8, device=dev)
+    best = ctypes.c_int32(-1)
+    times = (ctypes.c_float * max(count, 1))()
+    with torch.cuda.device(dev):
+        st = lib.sfp8_sparse_linear_search(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
+                                           _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w),
+                                           n, k, _ptr(bias), _ptr(out), _ptr(ws), ws.numel(),
+                                           _ptr(flush), 0 if flush is None else flush.numel(),
+                                           reps, ctypes.byref(best), times, count, _stream(dev))
+    _check(st, "sfp8_sparse_linear_search")
+    return int(best.value), [float(t) for t in times[:count]]
+
+
+def sfp8_sparse_linear_set_algo(m, n, k, algo, device=None):
+    with _dev_ctx(device):
+        st = load_library().sfp8_sparse_linear_set_algo(m, n, k, algo)
+    _check(st, "sfp8_sparse_linear_set_algo")
+
+
+def sfp8_sparse_linear_get_algo(m, n, k, device=None):
+    with _dev_ctx(device):
+        return int(load_library().sfp8_sparse_linear_get_algo(m, n, k))
 
 
 def sfp8_sparse_linear_quant_workspace_bytes(m, n, k, device=None):

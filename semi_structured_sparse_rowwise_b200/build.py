@@ -21,8 +21,6 @@ LIB_NAME = "libsfp8.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["sfp8_api.cu"]
-HEADERS = ["device_common.cuh", "quantize_rowwise.cuh", "sparse24_pack.cuh",
-           "sparse_linear.cuh"]
 
 
 def nvcc_path():
@@ -33,7 +31,8 @@ def nvcc_path():
 
 
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    headers = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
+    files = [os.path.join(CSRC, f) for f in SOURCES + headers]
     files.append(os.path.join(INCLUDE, "sfp8.h"))
     files.append(os.path.abspath(__file__))
     return files

@@ -130,7 +130,8 @@ __device__ __forceinline__ void prepare_chunk(const uint32_t* in, const uint32_t
     const uint32_t e = tab[idx];
     float f0, f1;
     G::kept(gw, e, f0, f1);
-    const uint32_t codes = cvt_pair<kFmt>(quotient_rn(f0, s, rcp), quotient_rn(f1, s, rcp));
+    const float2 t = quotient_rn2(make_float2(f0, f1), make_float2(-s, -s), make_float2(rcp, rcp));
+    const uint32_t codes = cvt_pair<kFmt>(t.x, t.y);
     zero_code = zero_code || (codes & 0x7Fu) == 0 || (codes & 0x7F00u) == 0;
     vals[g / 2] |= codes << (16 * (g % 2));
     meta |= ((e >> 16) & 0xFu) << (4 * g);

@@ -23,7 +23,9 @@
 // the codes are exactly those of the IEEE quotient (checked on the B200 for
 // every finite bf16 and fp16 x against the scale of every finite bf16 and
 // fp16 row amax, both formats, and for random fp32 x), with no branch and no
-// division per element.
+// division per element.  For 16-bit inputs the multiplies and fused
+// multiply-adds run two values at a time on sm_100's packed fp32x2
+// instructions.
 //
 // The kernels are launched as programmatic dependents: they let their own
 // dependents (the GEMM) launch at once, then wait for the preceding grid to
@@ -129,17 +131,41 @@ __device__ __forceinline__ float quotient_rn(float x, float s, float r) {
   return copysignf(t2, x);
 }
 
+// The same quotient for two values at once, on the packed fp32x2 pipe of
+// sm_100 (each lane an IEEE round-to-nearest multiply or fused multiply-add,
+// so the results are those of quotient_rn bit for bit).  fma(t, -s, x)
+// equals fma(-t, s, x) exactly (negation is exact).
+__device__ __forceinline__ float2 quotient_rn2(float2 x, float2 s2n, float2 r2) {
+  const float2 t0 = __fmul2_rn(x, r2);
+  const float2 t1 = __ffma2_rn(__ffma2_rn(t0, s2n, x), r2, t0);
+  const float2 t2 = __ffma2_rn(__ffma2_rn(t1, s2n, x), r2, t1);
+  return make_float2(copysignf(t2.x, x.x), copysignf(t2.y, x.y));
+}
+
 // Quantises one 16-byte input vector (already widened to floats) into
 // kPerVec codes packed little-endian; s is the row scale, r = RN(1/s).
 template <int kFmt, int kPerVec>
 __device__ __forceinline__ void quantize_vec(const float (&f)[kPerVec], float s, float r,
                                              uint32_t (&out)[kPerVec / 4]) {
+  if constexpr (kPerVec == 8) {
+    // 16-bit inputs (issue-bound): the packed quotient
+    const float2 s2n = make_float2(-s, -s);
+    const float2 r2 = make_float2(r, r);
 #pragma unroll
-  for (int w = 0; w < kPerVec / 4; ++w) {
-    float t[4];
+    for (int w = 0; w < kPerVec / 4; ++w) {
+      const float2 a = quotient_rn2(make_float2(f[4 * w], f[4 * w + 1]), s2n, r2);
+      const float2 b = quotient_rn2(make_float2(f[4 * w + 2], f[4 * w + 3]), s2n, r2);
+      out[w] = cvt_pair<kFmt>(a.x, a.y) | (cvt_pair<kFmt>(b.x, b.y) << 16);
+    }
+  } else {
+    // fp32 inputs (bound by HBM; measured faster with the scalar form)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) t[i] = quotient_rn(f[4 * w + i], s, r);
-    out[w] = cvt_pair<kFmt>(t[0], t[1]) | (cvt_pair<kFmt>(t[2], t[3]) << 16);
+    for (int w = 0; w < kPerVec / 4; ++w) {
+      float t[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[i] = quotient_rn(f[4 * w + i], s, r);
+      out[w] = cvt_pair<kFmt>(t[0], t[1]) | (cvt_pair<kFmt>(t[2], t[3]) << 16);
+    }
   }
 }
 

@@ -7,11 +7,14 @@
 
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "sfp8.h"
 #include "device_common.cuh"
 #include "quantize_rowwise.cuh"
+#include "quantize_tensorwise.cuh"
 #include "sparse24_pack.cuh"
 #include "prepare_weight24.cuh"
 #include "sparse_linear.cuh"
@@ -25,9 +28,12 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
+  int index = 0;
   int num_sms = 0;
   bool smem_attr_set[32] = {};   // (BN, KS, RA) instantiations
   int pair_clusters[4] = {};     // co-resident pairs of the pair kernel by (KS, WT) (0: unknown)
+  int tw_blocks[12] = {};        // co-resident CTAs per SM of the tensor-wise quantiser (0: unknown)
+  long long l2_bytes = 0;
 };
 
 std::mutex g_mutex;
@@ -51,8 +57,12 @@ sfp8_status current_device(DeviceInfo** out) {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
       return SFP8_ERR_CUDA;
+    int l2 = 0;
+    if (cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess) return SFP8_ERR_CUDA;
     d.is_sm100 = (major == 10 && minor == 0);
+    d.index = dev;
     d.num_sms = sms;
+    d.l2_bytes = l2;
     d.probed = true;
   }
   if (!d.is_sm100) return SFP8_ERR_ARCH;
@@ -208,6 +218,84 @@ sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64
   return launch_quantize<T, SFP8_E5M2>(x, rows, cols, ld, q, scales, st);
 }
 
+// ------------------------------------------------------------------ tensor-wise quantise
+
+// Upper bound on co-resident CTAs per SM of the tensor-wise kernel (2048
+// threads per SM / kTwThreads); sizes the partials of the reduction mode.
+constexpr int kTwMaxBlocksPerSm = 2048 / kTwThreads;
+
+size_t tensorwise_workspace_bytes(int num_sms, sfp8_amax_mode mode) {
+  size_t b = kTwSyncWords * sizeof(unsigned int);
+  if (mode == SFP8_AMAX_REDUCE) b += sizeof(float) * static_cast<size_t>(num_sms) * kTwMaxBlocksPerSm;
+  return b;
+}
+
+template <typename T, int kFmt, bool kAtomic>
+sfp8_status launch_tensorwise_cfg(DeviceInfo* dev, int slot, const void* x, int64_t numel,
+                                  void* q, float* scale, void* workspace, cudaStream_t st) {
+  auto kern = quantize_tensorwise_kernel<T, kFmt, kAtomic>;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (dev->tw_blocks[slot] == 0) {
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTwThreads, 0) !=
+              cudaSuccess || per_sm < 1) {
+        cudaGetLastError();
+        return SFP8_ERR_CUDA;
+      }
+      dev->tw_blocks[slot] = per_sm < kTwMaxBlocksPerSm ? per_sm : kTwMaxBlocksPerSm;
+    }
+  }
+  constexpr int P = InputTraits<T>::kPerVec;
+  constexpr int64_t kTile = static_cast<int64_t>(kTwThreads) * kTwUnroll;
+  const int64_t nvec = numel / P;
+  const int64_t tiles = (nvec + kTile - 1) / kTile;
+  const int64_t max_grid = static_cast<int64_t>(dev->tw_blocks[slot]) * dev->num_sms;
+  int64_t grid = tiles < max_grid ? tiles : max_grid;
+  if (grid < 1) grid = 1;
+  const int64_t per_cta = tiles > 0 ? (tiles + grid - 1) / grid : 0;
+  if (per_cta > 0) grid = (tiles + per_cta - 1) / per_cta;
+  // Tiles per run that sweep 1 marks to stay in L2: half the L2 over all runs.
+  const int64_t tile_bytes = kTile * 16;
+  int64_t keep = dev->l2_bytes / 2 / (grid * tile_bytes);
+  if (keep < 1) keep = 1;
+  unsigned int* sync = static_cast<unsigned int*>(workspace);
+  float* partials = reinterpret_cast<float*>(sync + kTwSyncWords);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kTwThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  // Cooperative: every CTA is resident at once (the kernel's grid barrier
+  // needs that), or the launch fails.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(x), numel, static_cast<uint8_t*>(q),
+                         scale, sync, partials, per_cta, keep) != cudaSuccess) {
+    cudaGetLastError();
+    return SFP8_ERR_CUDA;
+  }
+  return SFP8_OK;
+}
+
+template <typename T>
+sfp8_status launch_tensorwise(DeviceInfo* dev, int dslot, const void* x, int64_t numel,
+                              void* q, sfp8_dtype q_dtype, float* scale, sfp8_amax_mode mode,
+                              void* workspace, cudaStream_t st) {
+  const int slot = dslot * 4 + (q_dtype == SFP8_E5M2 ? 2 : 0) + (mode == SFP8_AMAX_ATOMIC ? 1 : 0);
+  if (q_dtype == SFP8_E4M3) {
+    if (mode == SFP8_AMAX_ATOMIC)
+      return launch_tensorwise_cfg<T, SFP8_E4M3, true>(dev, slot, x, numel, q, scale, workspace, st);
+    return launch_tensorwise_cfg<T, SFP8_E4M3, false>(dev, slot, x, numel, q, scale, workspace, st);
+  }
+  if (mode == SFP8_AMAX_ATOMIC)
+    return launch_tensorwise_cfg<T, SFP8_E5M2, true>(dev, slot, x, numel, q, scale, workspace, st);
+  return launch_tensorwise_cfg<T, SFP8_E5M2, false>(dev, slot, x, numel, q, scale, workspace, st);
+}
+
 // ------------------------------------------------------------------ linear plan
 
 constexpr long long kResidentActMax = 96 * 1024;   // resident activation slice limit
@@ -259,26 +347,84 @@ constexpr int kPairStepsPerStage = 2;
 constexpr int kPairWeightTiles = 2;
 constexpr int kPairTwoTileMinSteps = 64;   // k >= 8192
 
-LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
-  LinearPlan pl{};
+// A work split of the GEMM (an "algorithm"): everything else in a plan
+// follows from it and the shape.
+struct LinearChoice {
+  int pair;    // 1: the CTA-pair kernel
+  int bn;      // tokens per tile
+  int ks;      // k steps per pipeline stage
+  int wt;      // pair kernel: weight tiles per CTA (1 or 2); 1 otherwise
+  int whole;   // one-CTA kernel: 1 whole tiles per CTA, 0 stream-K; 1 for pairs
+  bool operator==(const LinearChoice& o) const {
+    return pair == o.pair && bn == o.bn && ks == o.ks && wt == o.wt && whole == o.whole;
+  }
+};
+
+// Pair tile width from the token count: the fewest tiles of at most
+// kPairMaxTokens, split evenly (rounded up to the pair MMA's N granularity
+// of 32).
+int pair_bn_for(int64_t m) {
+  const int64_t mt = (m + kPairMaxTokens - 1) / kPairMaxTokens;
+  return static_cast<int>(((m + mt - 1) / mt + 31) / 32 * 32);
+}
+
+// The built-in rule.
+LinearChoice default_choice(int64_t m, int64_t n, int64_t k, int num_sms) {
+  LinearChoice c{};
+  const int k_steps = static_cast<int>(k / kStepK);
+  const long long n_tiles = (n + kTileN - 1) / kTileN;
   if (m >= kPairMinTokens) {
-    pl.pair = 1;
-    // Tokens per tile: the fewest tiles of at most kPairMaxTokens, split
-    // evenly (rounded up to the pair MMA's N granularity of 32).
-    const int64_t mt = (m + kPairMaxTokens - 1) / kPairMaxTokens;
-    pl.bn = static_cast<int>(((m + mt - 1) / mt + 31) / 32 * 32);
-    pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
-    pl.k_steps = static_cast<int>(k / kStepK);
-    pl.ks = (kPairStepsPerStage == 2 && pl.k_steps % 2 == 0) ? 2 : 1;
-    pl.units = pl.k_steps / pl.ks;
-    pl.n_tiles = (n + kTileN - 1) / kTileN;
+    c.pair = 1;
+    c.bn = pair_bn_for(m);
+    const int m_tiles = static_cast<int>((m + c.bn - 1) / c.bn);
+    c.ks = (kPairStepsPerStage == 2 && k_steps % 2 == 0) ? 2 : 1;
     // Two weight tiles per CTA (512-row pair tiles) halve the activation
     // bytes per MMA, when that still leaves a tile for every pair.
     // The accumulators of a two-tile CTA are single-buffered (the epilogue
     // stalls the MMAs once per tile), so this pays off only for long k.
-    const long long groups2 = (pl.n_tiles + 3) / 4;
-    pl.wt = (kPairWeightTiles == 2 && pl.k_steps >= kPairTwoTileMinSteps &&
-             groups2 * pl.m_tiles >= num_sms / 2) ? 2 : 1;
+    const long long groups2 = (n_tiles + 3) / 4;
+    c.wt = (kPairWeightTiles == 2 && k_steps >= kPairTwoTileMinSteps &&
+            groups2 * m_tiles >= num_sms / 2) ? 2 : 1;
+    c.whole = 1;
+    return c;
+  }
+  c.pair = 0;
+  c.wt = 1;
+  c.bn = choose_bn(m);
+  // Several k steps per stage (20-50 KB): the stages are consumed in order,
+  // and fewer, larger copies keep more bytes in flight per SM than many
+  // small ones (measured on B200: the feed rate per SM grows with the copy
+  // size at a fixed shared-memory ring).
+  c.ks = (c.bn <= 32 && k_steps % 4 == 0) ? 4 : (c.bn <= 128 && k_steps % 2 == 0) ? 2 : 1;
+  const long long tiles = n_tiles * ((m + c.bn - 1) / c.bn);
+  if (c.bn <= 32) {
+    // Bandwidth-bound: whole tiles (no split-K fix-up) once there are enough
+    // of them to keep three quarters of the SMs streaming.
+    c.whole = tiles * 4 >= 3LL * num_sms ? 1 : 0;
+  } else {
+    // Compute-bound: whole tiles when the last wave is nearly full, or when
+    // one wave keeps three quarters of the SMs busy (measured with the
+    // search: m = 128, n = 14336, k = 4096 takes 25.6 us on 112 whole
+    // tiles, 37.9 us split over 148 SMs).
+    const long long waves = (tiles + num_sms - 1) / num_sms;
+    c.whole = ((tiles >= num_sms && tiles * 10 >= 9 * waves * num_sms) ||
+               (tiles < num_sms && tiles * 4 >= 3LL * num_sms)) ? 1 : 0;
+  }
+  return c;
+}
+
+// The plan of a choice (any choice from linear_choices is valid).
+LinearPlan plan_from_choice(int64_t m, int64_t n, int64_t k, int num_sms, const LinearChoice& c) {
+  LinearPlan pl{};
+  pl.bn = c.bn;
+  pl.ks = c.ks;
+  pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
+  pl.k_steps = static_cast<int>(k / kStepK);
+  pl.units = pl.k_steps / pl.ks;
+  pl.n_tiles = (n + kTileN - 1) / kTileN;
+  if (c.pair) {
+    pl.pair = 1;
+    pl.wt = c.wt;
     pl.tiles = ((pl.n_tiles + 2 * pl.wt - 1) / (2 * pl.wt)) * pl.m_tiles;
     pl.iters = pl.tiles * pl.units;
     pl.whole_tiles = 1;
@@ -291,28 +437,10 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
     pl.grid = 2 * static_cast<int>(pl.tiles < num_sms / 2 ? pl.tiles : num_sms / 2);
     return pl;
   }
-  pl.bn = choose_bn(m);
-  pl.m_tiles = static_cast<int>((m + pl.bn - 1) / pl.bn);
-  pl.k_steps = static_cast<int>(k / kStepK);
-  // Several k steps per stage (20-50 KB): the stages are consumed in order,
-  // and fewer, larger copies keep more bytes in flight per SM than many
-  // small ones (measured on B200: the feed rate per SM grows with the copy
-  // size at a fixed shared-memory ring).
-  pl.ks = (pl.bn <= 32 && pl.k_steps % 4 == 0) ? 4
-        : (pl.bn <= 128 && pl.k_steps % 2 == 0) ? 2 : 1;
-  pl.units = pl.k_steps / pl.ks;
-  pl.n_tiles = (n + kTileN - 1) / kTileN;
+  pl.wt = 1;
   pl.tiles = pl.n_tiles * pl.m_tiles;
   pl.iters = pl.tiles * pl.units;
-  if (pl.bn <= 32) {
-    // Bandwidth-bound: whole tiles (no split-K fix-up) once there are enough
-    // of them to keep three quarters of the SMs streaming.
-    pl.whole_tiles = pl.tiles * 4 >= 3LL * num_sms ? 1 : 0;
-  } else {
-    // Compute-bound: whole tiles when the last wave is nearly full.
-    const long long waves = (pl.tiles + num_sms - 1) / num_sms;
-    pl.whole_tiles = (pl.tiles >= num_sms && pl.tiles * 10 >= 9 * waves * num_sms) ? 1 : 0;
-  }
+  pl.whole_tiles = c.whole;
   // One token tile: keep the CTA's whole activation slice in shared memory
   // (one copy) when it is small; every stage is then one weight copy.
   const long long a_slice = static_cast<long long>(pl.bn) * k;
@@ -337,6 +465,69 @@ LinearPlan make_plan(int64_t m, int64_t n, int64_t k, int num_sms) {
     pl.counter_bytes = static_cast<size_t>(pl.tiles) * 4 * sizeof(unsigned int);
   }
   return pl;
+}
+
+constexpr int kMaxLinearChoices = 64;
+
+// Every work split offered for a shape: index 0 is the built-in rule, then
+// (without repeats) the one-CTA kernel at each tile width up to about twice
+// the token count, k steps per stage and whole-tile / stream-K split, and,
+// from 256 tokens, the CTA-pair kernel at tile widths 128..224, one or two
+// k steps per stage, one or two weight tiles per CTA.
+int linear_choices(int64_t m, int64_t n, int64_t k, int num_sms, LinearChoice* out) {
+  int count = 0;
+  auto add = [&](const LinearChoice& c) {
+    for (int i = 0; i < count; ++i)
+      if (out[i] == c) return;
+    if (count < kMaxLinearChoices) out[count++] = c;
+  };
+  add(default_choice(m, n, k, num_sms));
+  const int k_steps = static_cast<int>(k / kStepK);
+  for (int bn : {16, 32, 64, 128}) {
+    if (bn > 16 && bn >= 2 * m) continue;
+    for (int ks : {1, 2, 4}) {
+      if (k_steps % ks != 0 || (ks == 4 && bn > 32)) continue;
+      for (int whole : {1, 0}) add(LinearChoice{0, bn, ks, 1, whole});
+    }
+  }
+  if (m >= 256) {
+    const int m32 = static_cast<int>((m + 31) / 32 * 32);
+    for (int bn : {pair_bn_for(m), 128, 160, 192, 224}) {
+      if (bn > kPairMaxTokens || bn > m32) continue;
+      for (int ks : {1, 2}) {
+        if (k_steps % ks != 0) continue;
+        for (int wt : {1, 2}) add(LinearChoice{1, bn, ks, wt, 1});
+      }
+    }
+  }
+  return count;
+}
+
+// Shape-keyed choices set by sfp8_sparse_linear_set_algo, per device.
+struct AlgoEntry {
+  int64_t m, n, k;
+  int algo;
+  LinearChoice choice;
+};
+std::mutex g_algo_mutex;
+std::vector<AlgoEntry> g_algo_table[kMaxDevices];
+
+bool lookup_algo(int dev, int64_t m, int64_t n, int64_t k, AlgoEntry* e) {
+  std::lock_guard<std::mutex> lock(g_algo_mutex);
+  for (const AlgoEntry& a : g_algo_table[dev])
+    if (a.m == m && a.n == n && a.k == k) {
+      *e = a;
+      return true;
+    }
+  return false;
+}
+
+// The plan used by sfp8_sparse_linear on device `dev`: the table's choice
+// for this shape, else the built-in rule.
+LinearPlan make_plan(int dev, int64_t m, int64_t n, int64_t k, int num_sms) {
+  AlgoEntry e;
+  if (dev >= 0 && dev < kMaxDevices && lookup_algo(dev, m, n, k, &e)) return plan_from_choice(m, n, k, num_sms, e.choice);
+  return plan_from_choice(m, n, k, num_sms, default_choice(m, n, k, num_sms));
 }
 
 template <int BN, int KS, bool RA>
@@ -436,7 +627,7 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
     return SFP8_ERR_MISALIGNED;
   sfp8_status s = current_device(dev);
   if (s != SFP8_OK) return s;
-  *plan = make_plan(m, n, k, (*dev)->num_sms);
+  *plan = make_plan((*dev)->index, m, n, k, (*dev)->num_sms);
   return SFP8_OK;
 }
 
@@ -665,6 +856,42 @@ sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype, int64_t row
   }
 }
 
+size_t sfp8_quantize_tensorwise_workspace_bytes(sfp8_amax_mode mode) {
+  if (mode != SFP8_AMAX_REDUCE && mode != SFP8_AMAX_ATOMIC) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return tensorwise_workspace_bytes(sms, mode);
+}
+
+sfp8_status sfp8_quantize_tensorwise(const void* x, sfp8_dtype x_dtype, int64_t numel, void* q,
+                                     sfp8_dtype q_dtype, float* scale, sfp8_amax_mode mode,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!is_wide(x_dtype) || !is_fp8(q_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (mode != SFP8_AMAX_REDUCE && mode != SFP8_AMAX_ATOMIC) return SFP8_ERR_INVALID_ARG;
+  if (numel < 0) return SFP8_ERR_INVALID_ARG;
+  if (numel >= (int64_t(1) << 40)) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (scale == nullptr || workspace == nullptr || (numel > 0 && (x == nullptr || q == nullptr)))
+    return SFP8_ERR_INVALID_ARG;
+  if ((numel > 0 && (!aligned(x, 16) || !aligned(q, 16))) || !aligned(scale, 4) ||
+      !aligned(workspace, 16))
+    return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  if (workspace_bytes < tensorwise_workspace_bytes(dev->num_sms, mode)) return SFP8_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (x_dtype) {
+    case SFP8_BF16:
+      return launch_tensorwise<__nv_bfloat16>(dev, 0, x, numel, q, q_dtype, scale, mode, workspace, st);
+    case SFP8_F16:
+      return launch_tensorwise<__half>(dev, 1, x, numel, q, q_dtype, scale, mode, workspace, st);
+    default:
+      return launch_tensorwise<float>(dev, 2, x, numel, q, q_dtype, scale, mode, workspace, st);
+  }
+}
+
 sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows, int64_t cols,
                           int64_t ld, void* out, void* stream) {
   if (!is_wide(dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
@@ -791,7 +1018,7 @@ size_t sfp8_sparse_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 0;
-  const LinearPlan pl = make_plan(m, n, k, sms);
+  const LinearPlan pl = make_plan(dev, m, n, k, sms);
   return pl.partial_bytes + pl.counter_bytes;
 }
 
@@ -825,13 +1052,206 @@ sfp8_status sfp8_sparse_linear(const void* a_q, sfp8_dtype a_dtype, const float*
                        partials, counters, static_cast<cudaStream_t>(stream));
 }
 
+// ---- work-split selection ("algorithms")
+
+// Shape check shared by the algorithm entry points (no pointers involved).
+static bool algo_shape_ok(int64_t m, int64_t n, int64_t k) {
+  return m > 0 && n > 0 && k > 0 && k % kStepK == 0 && m < (int64_t(1) << 31) &&
+         n < (int64_t(1) << 31) && k < (int64_t(1) << 31);
+}
+
+int sfp8_sparse_linear_algo_count(int64_t m, int64_t n, int64_t k) {
+  if (!algo_shape_ok(m, n, k)) return 0;
+  DeviceInfo* dev = nullptr;
+  if (current_device(&dev) != SFP8_OK) return 0;
+  LinearChoice ch[kMaxLinearChoices];
+  return linear_choices(m, n, k, dev->num_sms, ch);
+}
+
+sfp8_status sfp8_sparse_linear_algo_info(int64_t m, int64_t n, int64_t k, int algo,
+                                         int32_t* info) {
+  if (info == nullptr || !algo_shape_ok(m, n, k)) return SFP8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  if (algo < 0 || algo >= count) return SFP8_ERR_INVALID_ARG;
+  const LinearPlan pl = plan_from_choice(m, n, k, dev->num_sms, ch[algo]);
+  info[0] = pl.pair;
+  info[1] = pl.bn;
+  info[2] = pl.ks;
+  info[3] = pl.wt;
+  info[4] = pl.whole_tiles;
+  info[5] = pl.ra;
+  info[6] = pl.stages;
+  info[7] = pl.grid;
+  return SFP8_OK;
+}
+
+size_t sfp8_sparse_linear_algo_workspace_bytes(int64_t m, int64_t n, int64_t k, int algo) {
+  if (!algo_shape_ok(m, n, k)) return 0;
+  DeviceInfo* dev = nullptr;
+  if (current_device(&dev) != SFP8_OK) return 0;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  if (algo < 0 || algo >= count) return 0;
+  const LinearPlan pl = plan_from_choice(m, n, k, dev->num_sms, ch[algo]);
+  return pl.partial_bytes + pl.counter_bytes;
+}
+
+size_t sfp8_sparse_linear_search_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  if (!algo_shape_ok(m, n, k)) return 0;
+  DeviceInfo* dev = nullptr;
+  if (current_device(&dev) != SFP8_OK) return 0;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  size_t most = 0;
+  for (int i = 0; i < count; ++i) {
+    const LinearPlan pl = plan_from_choice(m, n, k, dev->num_sms, ch[i]);
+    most = std::max(most, pl.partial_bytes + pl.counter_bytes);
+  }
+  return most;
+}
+
+sfp8_status sfp8_sparse_linear_algo(const void* a_q, sfp8_dtype a_dtype, const float* s_a,
+                                    int64_t m, const void* packed, sfp8_dtype w_dtype,
+                                    const float* s_w, int64_t n, int64_t k, const void* bias,
+                                    void* y, int algo, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  DeviceInfo* dev = nullptr;
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK || empty) return s;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  if (algo < 0 || algo >= count) return SFP8_ERR_INVALID_ARG;
+  pl = plan_from_choice(m, n, k, dev->num_sms, ch[algo]);
+  const size_t need = pl.partial_bytes + pl.counter_bytes;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+  float* partials = static_cast<float*>(workspace);
+  unsigned int* counters = need > 0 ? reinterpret_cast<unsigned int*>(
+                                          static_cast<uint8_t*>(workspace) + pl.partial_bytes)
+                                    : nullptr;
+  return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                       partials, counters, static_cast<cudaStream_t>(stream));
+}
+
+sfp8_status sfp8_sparse_linear_set_algo(int64_t m, int64_t n, int64_t k, int algo) {
+  if (!algo_shape_ok(m, n, k)) return SFP8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  if (algo >= count) return SFP8_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_algo_mutex);
+  std::vector<AlgoEntry>& t = g_algo_table[dev->index];
+  t.erase(std::remove_if(t.begin(), t.end(),
+                         [&](const AlgoEntry& a) { return a.m == m && a.n == n && a.k == k; }),
+          t.end());
+  if (algo > 0) t.push_back(AlgoEntry{m, n, k, algo, ch[algo]});
+  return SFP8_OK;
+}
+
+int sfp8_sparse_linear_get_algo(int64_t m, int64_t n, int64_t k) {
+  int dev = 0;
+  if (!algo_shape_ok(m, n, k) || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
+      dev >= kMaxDevices)
+    return 0;
+  AlgoEntry e;
+  return lookup_algo(dev, m, n, k, &e) ? e.algo : 0;
+}
+
+sfp8_status sfp8_sparse_linear_search(const void* a_q, sfp8_dtype a_dtype, const float* s_a,
+                                      int64_t m, const void* packed, sfp8_dtype w_dtype,
+                                      const float* s_w, int64_t n, int64_t k, const void* bias,
+                                      void* y, void* workspace, size_t workspace_bytes,
+                                      void* flush, size_t flush_bytes, int reps,
+                                      int* best_algo, float* times_us, int times_len,
+                                      void* stream) {
+  if (best_algo == nullptr || reps < 1 || reps > 64 || (flush == nullptr && flush_bytes > 0) ||
+      (times_us == nullptr && times_len > 0) || times_len < 0)
+    return SFP8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK) return s;
+  if (empty) return SFP8_ERR_INVALID_ARG;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, dev->num_sms, ch);
+  size_t need = 0;
+  for (int i = 0; i < count; ++i) {
+    const LinearPlan p = plan_from_choice(m, n, k, dev->num_sms, ch[i]);
+    need = std::max(need, p.partial_bytes + p.counter_bytes);
+  }
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
+  if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[128];
+  int made = 0;
+  for (; made < 2 * reps; ++made)
+    if (cudaEventCreate(&ev[made]) != cudaSuccess) break;
+  auto finish = [&](sfp8_status r) {
+    for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+    if (r != SFP8_OK) cudaGetLastError();
+    return r;
+  };
+  if (made < 2 * reps) return finish(SFP8_ERR_CUDA);
+  int best = 0;
+  float best_t = 0.0f;
+  float ts[64];
+  for (int a = 0; a < count; ++a) {
+    const LinearPlan p = plan_from_choice(m, n, k, dev->num_sms, ch[a]);
+    const size_t w = p.partial_bytes + p.counter_bytes;
+    float* partials = static_cast<float*>(workspace);
+    unsigned int* counters = w > 0 ? reinterpret_cast<unsigned int*>(
+                                         static_cast<uint8_t*>(workspace) + p.partial_bytes)
+                                   : nullptr;
+    // counters must start at zero: another split's partials may lie there
+    if (w > 0 && cudaMemsetAsync(workspace, 0, w, st) != cudaSuccess)
+      return finish(SFP8_ERR_CUDA);
+    s = launch_linear(dev, p, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                      partials, counters, st);   // warm-up
+    if (s != SFP8_OK) return finish(s);
+    for (int r = 0; r < reps; ++r) {
+      if (flush_bytes > 0 && cudaMemsetAsync(flush, r & 0xff, flush_bytes, st) != cudaSuccess)
+        return finish(SFP8_ERR_CUDA);
+      if (cudaEventRecord(ev[2 * r], st) != cudaSuccess) return finish(SFP8_ERR_CUDA);
+      s = launch_linear(dev, p, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
+                        partials, counters, st);
+      if (s != SFP8_OK) return finish(s);
+      if (cudaEventRecord(ev[2 * r + 1], st) != cudaSuccess) return finish(SFP8_ERR_CUDA);
+    }
+    if (cudaEventSynchronize(ev[2 * reps - 1]) != cudaSuccess) return finish(SFP8_ERR_CUDA);
+    for (int r = 0; r < reps; ++r) {
+      if (cudaEventElapsedTime(&ts[r], ev[2 * r], ev[2 * r + 1]) != cudaSuccess)
+        return finish(SFP8_ERR_CUDA);
+    }
+    std::sort(ts, ts + reps);
+    const float med = ts[reps / 2] * 1000.0f;
+    if (a < times_len) times_us[a] = med;
+    if (a == 0 || med < best_t) {
+      best = a;
+      best_t = med;
+    }
+  }
+  *best_algo = best;
+  return finish(SFP8_OK);
+}
+
 size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   if (m <= 0 || n <= 0 || k <= 0 || k % kStepK != 0) return 0;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 0;
-  const LinearPlan pl = make_plan(m, n, k, sms);
+  const LinearPlan pl = make_plan(dev, m, n, k, sms);
   return pl.partial_bytes + pl.counter_bytes;
 }
 

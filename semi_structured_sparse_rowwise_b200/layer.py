@@ -53,6 +53,25 @@ class SparseFp8Linear:
             self._ws[m] = ws
         return ws
 
+    def autotune(self, x, reps=10, flush_bytes=256 << 20):
+        """Times every work split of the GEMM for x's token count on this
+        layer's weight (sfp8_sparse_linear_search; a flush_bytes write before
+        each timed launch evicts the operands from L2) and stores the fastest
+        in the library's shape-keyed table, which every later forward with
+        that token count -- of any layer of the same shape on this device --
+        uses.  Returns (best algorithm, median microseconds per algorithm)."""
+        m = x.shape[0]
+        a_q, s_a = B.sfp8_quantize_rowwise(x, self.a_dtype)
+        flush = None
+        if flush_bytes:
+            flush = torch.empty((flush_bytes,), dtype=torch.uint8, device=self.device)
+        best, times = B.sfp8_sparse_linear_search(a_q, self.a_dtype, s_a, self.packed,
+                                                  self.w_dtype, self.s_w, self.n, self.k,
+                                                  bias=self.bias, reps=reps, flush=flush)
+        B.sfp8_sparse_linear_set_algo(m, self.n, self.k, best, self.device)
+        self._ws.pop(m, None)       # the workspace size follows the algorithm
+        return best, times
+
     def forward(self, x, out=None):
         """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16.
 

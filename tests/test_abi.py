@@ -74,6 +74,21 @@ def test_quantize_validation_without_gpu(lib):
     assert q(FAKE, 0, 4, 16, 20, FAKE, 3, FAKE, None) == 3       # ld*2 % 16
 
 
+def test_quantize_tensorwise_validation_without_gpu(lib):
+    q = lib.sfp8_quantize_tensorwise
+    ws = 1 << 20
+    assert q(FAKE, 9, 64, FAKE, 3, FAKE, 0, FAKE, ws, None) == 4       # bad input dtype
+    assert q(FAKE, 0, 64, FAKE, 2, FAKE, 0, FAKE, ws, None) == 4       # f32 output
+    assert q(FAKE, 0, 64, FAKE, 3, FAKE, 2, FAKE, ws, None) == 1       # unknown mode
+    assert q(FAKE, 0, -1, FAKE, 3, FAKE, 0, FAKE, ws, None) == 1       # negative numel
+    assert q(None, 0, 64, FAKE, 3, FAKE, 0, FAKE, ws, None) == 1       # null x
+    assert q(FAKE, 0, 64, FAKE, 3, None, 0, FAKE, ws, None) == 1       # null scale
+    assert q(FAKE, 0, 64, FAKE, 3, FAKE, 1, None, ws, None) == 1       # null workspace
+    assert q(FAKE_ODD, 0, 64, FAKE, 3, FAKE, 0, FAKE, ws, None) == 3   # misaligned x
+    assert q(FAKE, 0, 64, FAKE_ODD, 3, FAKE, 0, FAKE, ws, None) == 3   # misaligned q
+    assert q(FAKE, 0, 1 << 41, FAKE, 3, FAKE, 0, FAKE, ws, None) == 2  # too large
+    assert lib.sfp8_quantize_tensorwise_workspace_bytes(7) == 0
+
 def test_prune_compress_validation_without_gpu(lib):
     assert lib.sfp8_prune_24(FAKE, 3, 4, 16, 16, FAKE, None) == 4
     assert lib.sfp8_prune_24(FAKE, 0, 4, 20, 20, FAKE, None) == 2
