@@ -550,9 +550,11 @@ def run_tensorwise(args):
     g = torch.Generator(device=dev).manual_seed(1004)
     reps = max(args.steps, 5)
     table = []
+    dtypes = {"f32": torch.float32, "bf16": torch.bfloat16}
+    sizes = [int(v) for v in args.tw_numel.split(",")] if args.tw_numel else TENSORWISE_SIZES
     with ClockSampler(local) as clk:
-        for dtype in (torch.float32, torch.bfloat16):
-            for numel in TENSORWISE_SIZES:
+        for dtype in [dtypes[d] for d in args.tw_dtype.split(",")]:
+            for numel in sizes:
                 x = torch.randn(numel, generator=g, device=dev, dtype=torch.float32).to(dtype)
                 q = torch.empty((numel,), dtype=torch.uint8, device=dev)
                 sc = torch.empty((1,), dtype=torch.float32, device=dev)
@@ -589,13 +591,13 @@ def run_tensorwise(args):
     st, flags = S.sfp8_read_device_status(clear=True)
     if st != 0:
         raise RuntimeError("device status %d flags %#x" % (st, flags))
-    big = [r for r in table if r["numel"] == TENSORWISE_SIZES[-1]]
+    big = [r for r in table if r["numel"] == max(sizes)]
     best = max(big, key=lambda r: r["GB/s"])
     line = {
         "metric": "tensor-wise FP8 quantise GB/s (one global amax)", "value": best["GB/s"],
         "unit": "GB/s", "n_gpus": world, "steps": reps, "warmup": args.warmup,
         "higher_is_better": True, "dtype": "e4m3", "data": "synthetic",
-        "config": {"workload": "quantize_tensorwise", "sizes": list(TENSORWISE_SIZES),
+        "config": {"workload": "quantize_tensorwise", "sizes": list(sizes),
                    "l2": "256 MB write before every timed call", "seed": 1004},
         "roofline": {"bound": "hbm", "achieved": best["GB/s"], "peak": peak, "unit": "GB/s",
                      "frac": best["GB/s"] / peak, "traffic": None,
@@ -621,6 +623,11 @@ def main():
                     "the standalone tensor-wise quantiser on the pages' conversion sizes")
     ap.add_argument("--shape", type=int, default=2, choices=[0, 1, 2, 3],
                     help="prefill_8b shape: 0 QKV, 1 O, 2 up (default), 3 down")
+    ap.add_argument("--tw-numel", default="",
+                    help="quantize_tensorwise: comma-separated element counts (default: the "
+                    "pages' 65500, 2^20, 2^24, 2^28)")
+    ap.add_argument("--tw-dtype", default="f32,bf16",
+                    help="quantize_tensorwise: input dtypes, comma-separated (f32, bf16)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--all-m", action="store_true", help="also time M=1 and M=4")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -338,8 +338,10 @@ int choose_bn(int64_t m) {
 // phases ahead of a slot, so the parity it waits on is unambiguous.
 int producers_for(int stages) { return stages < kPlanProducers ? stages : kPlanProducers; }
 
-// Token count from which the CTA-pair kernel is used.
+// Token count from which the CTA-pair kernel is used; from
+// kPairSmallMinTokens it is used when its tiles keep enough SMs busy.
 constexpr int64_t kPairMinTokens = 512;
+constexpr int64_t kPairSmallMinTokens = 256;
 // k steps per pipeline stage of the CTA-pair kernel (when k allows).
 constexpr int kPairStepsPerStage = 2;
 // Weight tiles per CTA of the CTA-pair kernel (when there are enough tiles
@@ -388,28 +390,49 @@ LinearChoice default_choice(int64_t m, int64_t n, int64_t k, int num_sms) {
     c.whole = 1;
     return c;
   }
+  // 256..511 tokens: CTA pairs when their tiles keep at least 60 % of the
+  // pairs busy -- two weight tiles per CTA first (each activation byte feeds
+  // twice the MMAs), then the widest token tile.
+  if (m >= kPairSmallMinTokens) {
+    for (int wt = 2; wt >= 1; --wt) {
+      for (int bn = pair_bn_for(m); bn >= 128; bn -= 32) {
+        const long long pairs = ((n_tiles + 2 * wt - 1) / (2 * wt)) * ((m + bn - 1) / bn);
+        if (pairs * 10 >= 6LL * (num_sms / 2)) {
+          c.pair = 1;
+          c.bn = bn;
+          c.ks = (k_steps % 2 == 0) ? 2 : 1;
+          c.wt = wt;
+          c.whole = 1;
+          return c;
+        }
+      }
+    }
+  }
   c.pair = 0;
   c.wt = 1;
-  c.bn = choose_bn(m);
   // Several k steps per stage (20-50 KB): the stages are consumed in order,
   // and fewer, larger copies keep more bytes in flight per SM than many
   // small ones (measured on B200: the feed rate per SM grows with the copy
   // size at a fixed shared-memory ring).
-  c.ks = (c.bn <= 32 && k_steps % 4 == 0) ? 4 : (c.bn <= 128 && k_steps % 2 == 0) ? 2 : 1;
-  const long long tiles = n_tiles * ((m + c.bn - 1) / c.bn);
-  if (c.bn <= 32) {
-    // Bandwidth-bound: whole tiles (no split-K fix-up) once there are enough
-    // of them to keep three quarters of the SMs streaming.
-    c.whole = tiles * 4 >= 3LL * num_sms ? 1 : 0;
-  } else {
-    // Compute-bound: whole tiles when the last wave is nearly full, or when
-    // one wave keeps three quarters of the SMs busy (measured with the
-    // search: m = 128, n = 14336, k = 4096 takes 25.6 us on 112 whole
-    // tiles, 37.9 us split over 148 SMs).
-    const long long waves = (tiles + num_sms - 1) / num_sms;
-    c.whole = ((tiles >= num_sms && tiles * 10 >= 9 * waves * num_sms) ||
-               (tiles < num_sms && tiles * 4 >= 3LL * num_sms)) ? 1 : 0;
+  auto ks_for = [&](int bn) {
+    return (bn <= 32 && k_steps % 4 == 0) ? 4 : (bn <= 128 && k_steps % 2 == 0) ? 2 : 1;
+  };
+  // Whole tiles (no split-K fix-up) with the widest token tile that keeps
+  // three quarters of the SMs busy: narrower tiles re-read the weight from L2
+  // once per token tile, which costs less than idle SMs or a split.
+  for (int bn = choose_bn(m); bn >= 16; bn /= 2) {
+    const long long tiles = n_tiles * ((m + bn - 1) / bn);
+    if (tiles * 4 >= 3LL * num_sms) {
+      c.bn = bn;
+      c.ks = ks_for(bn);
+      c.whole = 1;
+      return c;
+    }
   }
+  // Too few tiles even at 16 tokens: split the k range over the SMs.
+  c.bn = choose_bn(m);
+  c.ks = ks_for(c.bn);
+  c.whole = 0;
   return c;
 }
 
