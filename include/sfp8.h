@@ -419,6 +419,16 @@ sfp8_status sfp8_sparse_linear_noalloc(const void* a_q, sfp8_dtype a_dtype,
                                        void* y, void* stream);
 
 /*
+ * Test of the failure path (no counterpart on the pages): launches one
+ * thread that waits, with the same bounded wait as every pipeline of this
+ * library, on a barrier that nothing completes.  After the wait limit (about
+ * a second) it sets SFP8_DEVICE_TIMEOUT in the status word and returns; no
+ * fault, nothing left in flight, the context stays usable.  Read and clear
+ * the word with sfp8_read_device_status afterwards.
+ */
+sfp8_status sfp8_selftest_timeout(void* stream);
+
+/*
  * Reads (and with clear != 0, resets) the current device's status word.
  * Synchronises the device first.  *flags receives SFP8_DEVICE_* bits.
  * Returns SFP8_ERR_TIMEOUT / SFP8_ERR_DEVICE_CHECK when such a bit is set,

@@ -19,7 +19,7 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_sparse_linear_search, sfp8_sparse_linear_set_algo,
                       sfp8_sparse_linear_get_algo,
                       sfp8_sparse_linear_quant, sfp8_sparse_linear_quant_workspace_bytes,
-                      new_quant_workspace, sfp8_read_device_status,
+                      new_quant_workspace, sfp8_read_device_status, sfp8_selftest_timeout,
                       sfp8_status_string, sfp8_layout_version)
 from .layer import SparseFp8Linear
 
@@ -36,6 +36,6 @@ __all__ = [
     "sfp8_sparse_linear_algo", "sfp8_sparse_linear_search", "sfp8_sparse_linear_set_algo",
     "sfp8_sparse_linear_get_algo",
     "sfp8_sparse_linear_quant_workspace_bytes", "new_quant_workspace",
-    "sfp8_read_device_status", "sfp8_status_string",
+    "sfp8_read_device_status", "sfp8_selftest_timeout", "sfp8_status_string",
     "sfp8_layout_version", "SparseFp8Linear",
 ]

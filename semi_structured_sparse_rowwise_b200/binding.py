@@ -71,6 +71,7 @@ SIGNATURES = {
     "sfp8_sparse_linear_quant": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p, _c_void_p,
                                         _i64, _c_void_p, _i32, _c_void_p, _i64, _i64,
                                         _c_void_p, _c_void_p, _c_void_p, _sz, _c_void_p]),
+    "sfp8_selftest_timeout": (_i32, [_c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
     "sfp8_layout_version": (_i32, []),
@@ -478,6 +479,16 @@ def sfp8_sparse_linear_quant(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None, 
                                           workspace.numel(), _stream(dev))
     _check(st, "sfp8_sparse_linear_quant")
     return out, a_q, s_a
+
+
+def sfp8_selftest_timeout(device=None):
+    """Runs the library's failure-path self-test on `device` (a bounded wait
+    that runs out, about a second); read the status word afterwards."""
+    lib = load_library()
+    with _dev_ctx(device):
+        dev = torch.cuda.current_device()
+        st = lib.sfp8_selftest_timeout(_stream(dev))
+    _check(st, "sfp8_selftest_timeout")
 
 
 def sfp8_read_device_status(clear=True):

@@ -819,6 +819,28 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
 }  // namespace
 }  // namespace sfp8
 
+namespace sfp8 {
+namespace {
+
+// Self-test of the failure path: one thread waits, with the bounded wait of
+// every pipeline in this library, on an mbarrier that nothing arrives on.
+// After kWaitLimitCycles the wait gives up, records SFP8_DEVICE_TIMEOUT in
+// the status word and the kernel returns; nothing is left in flight.
+__global__ void selftest_wait_timeout_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag);
+}
+
+}  // namespace
+}  // namespace sfp8
+
 using namespace sfp8;
 
 extern "C" {
@@ -1312,6 +1334,14 @@ sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t 
   if (s != SFP8_OK) return s;
   return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
                        partials, counters, st);
+}
+
+sfp8_status sfp8_selftest_timeout(void* stream) {
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
 }
 
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
