@@ -292,6 +292,15 @@ int sfp8_sparse_linear_algo_count(int64_t m, int64_t n, int64_t k);
 sfp8_status sfp8_sparse_linear_algo_info(int64_t m, int64_t n, int64_t k, int algo,
                                          int32_t* info);
 
+/* The same list for a device of num_sms SMs without touching any device (a
+ * host-only query, e.g. to inspect plans offline): the count, and
+ * info[0..11] = {pair kernel, tokens per tile, k steps per stage, weight
+ * tiles per CTA, whole tiles, resident activation, stages, CTAs, producer
+ * warps, dynamic shared memory bytes, workspace bytes, token tiles}. */
+int sfp8_sparse_linear_plan_count(int64_t m, int64_t n, int64_t k, int num_sms);
+sfp8_status sfp8_sparse_linear_plan_info(int64_t m, int64_t n, int64_t k, int num_sms,
+                                         int algo, int64_t* info);
+
 /* Workspace bytes of one algorithm, and the most over all algorithms of the
  * shape (what sfp8_sparse_linear_search needs). */
 size_t sfp8_sparse_linear_algo_workspace_bytes(int64_t m, int64_t n, int64_t k, int algo);

@@ -56,6 +56,9 @@ SIGNATURES = {
     "sfp8_sparse_linear_algo_info": (_i32, [_i64, _i64, _i64, _i32,
                                             ctypes.POINTER(ctypes.c_int32)]),
     "sfp8_sparse_linear_algo_workspace_bytes": (_sz, [_i64, _i64, _i64, _i32]),
+    "sfp8_sparse_linear_plan_count": (_i32, [_i64, _i64, _i64, _i32]),
+    "sfp8_sparse_linear_plan_info": (_i32, [_i64, _i64, _i64, _i32, _i32,
+                                            ctypes.POINTER(ctypes.c_int64)]),
     "sfp8_sparse_linear_search_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "sfp8_sparse_linear_algo": (_i32, [_c_void_p, _i32, _c_void_p, _i64, _c_void_p, _i32,
                                        _c_void_p, _i64, _i64, _c_void_p, _c_void_p, _i32,
@@ -362,6 +365,23 @@ def sfp8_sparse_linear_algo_info(m, n, k, algo, device=None):
         st = load_library().sfp8_sparse_linear_algo_info(m, n, k, algo, info)
     _check(st, "sfp8_sparse_linear_algo_info")
     return dict(zip(ALGO_FIELDS, [int(v) for v in info]))
+
+
+PLAN_FIELDS = ("pair", "bn", "ks", "wt", "whole_tiles", "ra", "stages", "grid", "producers",
+               "smem_bytes", "workspace_bytes", "m_tiles")
+
+
+def sfp8_sparse_linear_plan(m, n, k, num_sms, algo=0):
+    """Host-only: the plan of an algorithm for a device of num_sms SMs (dict
+    of PLAN_FIELDS), no device involved."""
+    info = (ctypes.c_int64 * len(PLAN_FIELDS))()
+    st = load_library().sfp8_sparse_linear_plan_info(m, n, k, num_sms, algo, info)
+    _check(st, "sfp8_sparse_linear_plan_info")
+    return dict(zip(PLAN_FIELDS, [int(v) for v in info]))
+
+
+def sfp8_sparse_linear_plan_count(m, n, k, num_sms):
+    return int(load_library().sfp8_sparse_linear_plan_count(m, n, k, num_sms))
 
 
 def sfp8_sparse_linear_algo_workspace_bytes(m, n, k, algo, device=None):

@@ -1105,6 +1105,26 @@ static bool algo_shape_ok(int64_t m, int64_t n, int64_t k) {
          n < (int64_t(1) << 31) && k < (int64_t(1) << 31);
 }
 
+int sfp8_sparse_linear_plan_count(int64_t m, int64_t n, int64_t k, int num_sms) {
+  if (!algo_shape_ok(m, n, k) || num_sms < 2) return 0;
+  LinearChoice ch[kMaxLinearChoices];
+  return linear_choices(m, n, k, num_sms, ch);
+}
+
+sfp8_status sfp8_sparse_linear_plan_info(int64_t m, int64_t n, int64_t k, int num_sms, int algo,
+                                         int64_t* info) {
+  if (info == nullptr || !algo_shape_ok(m, n, k) || num_sms < 2) return SFP8_ERR_INVALID_ARG;
+  LinearChoice ch[kMaxLinearChoices];
+  const int count = linear_choices(m, n, k, num_sms, ch);
+  if (algo < 0 || algo >= count) return SFP8_ERR_INVALID_ARG;
+  const LinearPlan pl = plan_from_choice(m, n, k, num_sms, ch[algo]);
+  const int64_t v[12] = {pl.pair, pl.bn, pl.ks, pl.wt, pl.whole_tiles, pl.ra, pl.stages,
+                         pl.grid, pl.producers, pl.smem_bytes,
+                         static_cast<int64_t>(pl.partial_bytes + pl.counter_bytes), pl.m_tiles};
+  for (int i = 0; i < 12; ++i) info[i] = v[i];
+  return SFP8_OK;
+}
+
 int sfp8_sparse_linear_algo_count(int64_t m, int64_t n, int64_t k) {
   if (!algo_shape_ok(m, n, k)) return 0;
   DeviceInfo* dev = nullptr;
