@@ -386,6 +386,29 @@ sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t 
                                      size_t workspace_bytes, void* stream);
 
 /*
+ * The layer's forward from host memory to host memory in one call: on
+ * `stream`, the copy of x_host into the device staging buffer x_dev, then
+ * exactly sfp8_sparse_linear_quant on it, then the copy of y_dev into y_host.
+ * For the end-to-end path of a caller that holds its activations on the
+ * host; with page-locked host buffers the copies are asynchronous like the
+ * rest (pageable buffers work, and make the copies synchronous).
+ *
+ *  x_host  host, [m, k] of x_dtype, contiguous.
+ *  x_dev   device, [m, k] of x_dtype, contiguous, 16-byte aligned (staging).
+ *  y_dev   device, [m, n] bf16 (as y of sfp8_sparse_linear).
+ *  y_host  host, [m, n] bf16, contiguous, written.
+ *  Everything else as for sfp8_sparse_linear_quant (ld_x = k).  All
+ *  arguments are validated before anything is enqueued.
+ */
+sfp8_status sfp8_sparse_linear_quant_host(const void* x_host, void* x_dev, sfp8_dtype x_dtype,
+                                          sfp8_dtype a_dtype, void* a_q, float* s_a,
+                                          int64_t m, const void* packed, sfp8_dtype w_dtype,
+                                          const float* s_w, int64_t n, int64_t k,
+                                          const void* bias, void* y_dev, void* y_host,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream);
+
+/*
  * Size of the scratch buffer built into the library for
  * sfp8_sparse_linear_noalloc (per device that loads the library).
  */

@@ -21,7 +21,7 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_sparse_linear_quant, sfp8_sparse_linear_quant_workspace_bytes,
                       new_quant_workspace, sfp8_read_device_status, sfp8_selftest_timeout,
                       sfp8_status_string, sfp8_layout_version)
-from .layer import SparseFp8Linear
+from .layer import HostPipeline, SparseFp8Linear
 
 __all__ = [
     "Sfp8Error", "load_library", "library_path", "new_workspace",
@@ -37,5 +37,5 @@ __all__ = [
     "sfp8_sparse_linear_get_algo",
     "sfp8_sparse_linear_quant_workspace_bytes", "new_quant_workspace",
     "sfp8_read_device_status", "sfp8_selftest_timeout", "sfp8_status_string",
-    "sfp8_layout_version", "SparseFp8Linear",
+    "sfp8_layout_version", "SparseFp8Linear", "HostPipeline",
 ]

@@ -75,6 +75,10 @@ SIGNATURES = {
                                         _i64, _c_void_p, _i32, _c_void_p, _i64, _i64,
                                         _c_void_p, _c_void_p, _c_void_p, _sz, _c_void_p]),
     "sfp8_selftest_timeout": (_i32, [_c_void_p]),
+    "sfp8_sparse_linear_quant_host": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _c_void_p,
+                                             _c_void_p, _i64, _c_void_p, _i32, _c_void_p, _i64,
+                                             _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                             _sz, _c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
     "sfp8_layout_version": (_i32, []),
@@ -509,6 +513,33 @@ def sfp8_selftest_timeout(device=None):
         dev = torch.cuda.current_device()
         st = lib.sfp8_selftest_timeout(_stream(dev))
     _check(st, "sfp8_selftest_timeout")
+
+
+def sfp8_sparse_linear_quant_host(x_host, a_dtype, packed, w_dtype, s_w, n, k, x_dev, a_q, s_a,
+                                  y_dev, y_host, workspace, bias=None):
+    """Host x [m, k] -> host y [m, n] in one library call: copy in, quantise,
+    sparse linear, copy out, all on the current stream (page-locked host
+    tensors keep it asynchronous).  Every buffer is given by the caller."""
+    lib = load_library()
+    _require_cuda(x_dev, a_q, s_a, packed, s_w, bias, y_dev, workspace)
+    if x_host.is_cuda or y_host.is_cuda:
+        raise ValueError("x_host and y_host must be host tensors")
+    if not (x_host.is_contiguous() and y_host.is_contiguous() and x_dev.is_contiguous()):
+        raise ValueError("x_host, x_dev and y_host must be contiguous")
+    m = x_host.shape[0]
+    if x_host.shape != (m, k) or x_dev.shape != (m, k) or y_host.shape != (m, n):
+        raise ValueError("shapes: x_host/x_dev [m, k], y_host [m, n]")
+    xd = TORCH_WIDE.get(x_host.dtype)
+    if xd is None or x_dev.dtype != x_host.dtype or y_host.dtype != torch.bfloat16:
+        raise ValueError("x dtype bfloat16/float16/float32 (same on host and device), y bfloat16")
+    dev = x_dev.device
+    with torch.cuda.device(dev):
+        st = lib.sfp8_sparse_linear_quant_host(
+            _ptr(x_host), _ptr(x_dev), DTYPE[xd], DTYPE[_fp8_name(a_dtype)], _ptr(a_q), _ptr(s_a),
+            m, _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n, k, _ptr(bias), _ptr(y_dev),
+            _ptr(y_host), _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(st, "sfp8_sparse_linear_quant_host")
+    return y_host
 
 
 def sfp8_read_device_status(clear=True):

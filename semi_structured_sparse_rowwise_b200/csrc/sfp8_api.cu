@@ -1364,6 +1364,46 @@ sfp8_status sfp8_selftest_timeout(void* stream) {
   return launch_status();
 }
 
+sfp8_status sfp8_sparse_linear_quant_host(const void* x_host, void* x_dev, sfp8_dtype x_dtype,
+                                          sfp8_dtype a_dtype, void* a_q, float* s_a, int64_t m,
+                                          const void* packed, sfp8_dtype w_dtype,
+                                          const float* s_w, int64_t n, int64_t k,
+                                          const void* bias, void* y_dev, void* y_host,
+                                          void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  if (!is_wide(x_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  DeviceInfo* dev = nullptr;
+  LinearPlan pl{};
+  bool empty = false;
+  sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y_dev,
+                                  &dev, &pl, &empty);
+  if (s != SFP8_OK) return s;
+  if (m == 0) return SFP8_OK;
+  if (x_host == nullptr || x_dev == nullptr || (n > 0 && y_host == nullptr))
+    return SFP8_ERR_INVALID_ARG;
+  if (!aligned(x_dev, 16)) return SFP8_ERR_MISALIGNED;
+  if (!empty) {
+    const size_t need = pl.partial_bytes + pl.counter_bytes;
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
+    if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t x_bytes = static_cast<size_t>(m) * static_cast<size_t>(k) * elem_size(x_dtype);
+  if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SFP8_ERR_CUDA;
+  }
+  s = sfp8_sparse_linear_quant(x_dev, x_dtype, k, a_dtype, a_q, s_a, m, packed, w_dtype, s_w, n,
+                               k, bias, y_dev, workspace, workspace_bytes, stream);
+  if (s != SFP8_OK || n == 0) return s;
+  const size_t y_bytes = static_cast<size_t>(m) * static_cast<size_t>(n) * 2;
+  if (cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SFP8_ERR_CUDA;
+  }
+  return SFP8_OK;
+}
+
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {
   if (flags == nullptr) return SFP8_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return SFP8_ERR_CUDA;

@@ -89,6 +89,13 @@ def test_quantize_tensorwise_validation_without_gpu(lib):
     assert q(FAKE, 0, 1 << 41, FAKE, 3, FAKE, 0, FAKE, ws, None) == 2  # too large
     assert lib.sfp8_quantize_tensorwise_workspace_bytes(7) == 0
 
+
+def test_host_path_validation_without_gpu(lib):
+    f = lib.sfp8_sparse_linear_quant_host
+    # an fp8 activation input is rejected before any device is touched
+    assert f(FAKE, FAKE, 3, 3, FAKE, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE,
+             FAKE, 0, None) == 4
+
 def test_prune_compress_validation_without_gpu(lib):
     assert lib.sfp8_prune_24(FAKE, 3, 4, 16, 16, FAKE, None) == 4
     assert lib.sfp8_prune_24(FAKE, 0, 4, 20, 20, FAKE, None) == 2

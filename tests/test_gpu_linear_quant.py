@@ -112,3 +112,59 @@ def test_zero_outputs_still_quantises():
     torch.cuda.synchronize()
     assert y.shape == (8, 0)
     assert torch.equal(aq, aq2) and torch.equal(sa.view(torch.int32), sa2.view(torch.int32))
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_path_matches_device_path(pinned):
+    """sfp8_sparse_linear_quant_host (copy in, quantise, linear, copy out in
+    one call) gives the device path's bits, from page-locked or pageable host
+    buffers, on repeated calls."""
+    m, k, n = 16, 1024, 700
+    x = synthetic.activation(8100, m, k, dist="student_t3")
+    w = synthetic.weight(8101, n, k)
+    b = synthetic.bias(8102, n)
+    layer = S.SparseFp8Linear(bf16_dev(w), bias=bf16_dev(b).float())
+    x_host = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    y_host = torch.empty((m, n), dtype=torch.bfloat16)
+    if pinned:
+        x_host, y_host = x_host.pin_memory(), y_host.pin_memory()
+    y_dev = layer(x_host.cuda())
+    for _ in range(3):
+        y_host.fill_(float("nan"))
+        layer.forward_host(x_host, y_host)
+        torch.cuda.synchronize()
+        assert torch.equal(y_host.view(torch.int16), y_dev.cpu().view(torch.int16))
+    st, flags = S.sfp8_read_device_status(clear=True)
+    assert st == 0 and flags == 0
+
+
+def test_host_pipeline_eager_and_captured():
+    """HostPipeline: copies in, forward and copies out on three streams with
+    rotating buffers; each batch's y_host equals the device path's bits, both
+    for eager submits and for a captured graph replayed twice."""
+    m, k, n = 16, 512, 300
+    w = synthetic.weight(8200, n, k)
+    layer = S.SparseFp8Linear(bf16_dev(w))
+    xs = [synthetic.activation(8201 + i, m, k, dist="student_t3") for i in range(5)]
+    x_hosts = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+               .pin_memory() for x in xs]
+    refs = [layer(xh.cuda()).cpu() for xh in x_hosts]
+    y_hosts = [torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for _ in xs]
+    pipe = S.HostPipeline(layer, m, depth=3)
+    for xh, yh in zip(x_hosts, y_hosts):
+        pipe.submit(xh, yh)
+    pipe.synchronize()
+    for yh, ref in zip(y_hosts, refs):
+        assert torch.equal(yh.view(torch.int16), ref.view(torch.int16))
+    pipe2 = S.HostPipeline(layer, m, depth=2)
+    g = pipe2.capture(x_hosts, y_hosts)
+    for _ in range(2):
+        for yh in y_hosts:
+            yh.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for yh, ref in zip(y_hosts, refs):
+            assert torch.equal(yh.view(torch.int16), ref.view(torch.int16))
+    del g
+    st, flags = S.sfp8_read_device_status(clear=True)
+    assert st == 0 and flags == 0
