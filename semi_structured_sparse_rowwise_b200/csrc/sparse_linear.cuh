@@ -387,8 +387,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t a_addr =
                 RA ? smem_u32(ra_base) + (u * KS + j) * Cfg::kATileBytes
                    : st + KS * kWTileBytes + j * Cfg::kATileBytes;
-            // metadata: 128 rows x 16 bytes, no swizzle, 8-row groups 128 B apart
-            tc_cp_128x128b(e_tmem + 4 * j, smem_desc(e_addr, 0, 128, kNoSwizzle));
+            // metadata: 128 rows x 16 bytes, no swizzle, 8-row groups 128 B apart;
+            // k steps j and j + 1 (consecutive tiles, kWTileBytes apart) in one
+            // 128 x 256-bit copy
+            if constexpr (KS == 1) {
+              tc_cp_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kNoSwizzle));
+            } else if (j % 2 == 0) {
+              tc_cp_128x256b(e_tmem + 4 * j, smem_desc(e_addr, kWTileBytes, 128, kNoSwizzle));
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               // weight: 128 rows x 64 B (64B swizzle, 8-row atoms 512 B apart);

@@ -273,7 +273,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
               const uint32_t w_addr = st + (h * KS + j) * kWTileBytes;
               const uint32_t e_col = e_tmem + 4 * (h * KS + j);
               const uint32_t d_tmem = tmem_base + (WT == 1 ? acc : h) * kPairMaxTokens;
-              tc_cp_128x128b_pair(e_col, smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
+              // metadata of k steps j and j + 1 of this slot (consecutive tiles)
+              // in one 128 x 256-bit copy
+              if constexpr (KS == 1) {
+                tc_cp_128x128b_pair(e_col, smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
+              } else if (j % 2 == 0) {
+                tc_cp_128x256b_pair(e_col, smem_desc(w_addr + kWValBytes, kWTileBytes, 128,
+                                                     kNoSwizzle));
+              }
 #pragma unroll
               for (int kh = 0; kh < 2; ++kh) {
                 const uint64_t adesc = smem_desc(w_addr + 32 * kh, 16, 512, kSwizzle64);
