@@ -494,9 +494,10 @@ constexpr int kMaxLinearChoices = 64;
 
 // Every work split offered for a shape: index 0 is the built-in rule, then
 // (without repeats) the one-CTA kernel at each tile width up to about twice
-// the token count, k steps per stage and whole-tile / stream-K split, and,
-// from 256 tokens, the CTA-pair kernel at tile widths 128..224, one or two
-// k steps per stage, one or two weight tiles per CTA.
+// the token count, k steps per stage and whole-tile / stream-K split, and
+// the CTA-pair kernel at tile widths up to the token count rounded up to 32
+// (128..224 from 256 tokens), one or two k steps per stage, one or two
+// weight tiles per CTA.
 int linear_choices(int64_t m, int64_t n, int64_t k, int num_sms, LinearChoice* out) {
   int count = 0;
   auto add = [&](const LinearChoice& c) {
@@ -513,10 +514,12 @@ int linear_choices(int64_t m, int64_t n, int64_t k, int num_sms, LinearChoice* o
       for (int whole : {1, 0}) add(LinearChoice{0, bn, ks, 1, whole});
     }
   }
-  if (m >= 256) {
+  {
+    // CTA pairs at every token count: from 256 tokens the tile widths
+    // 128..224; below, the widths up to the token count rounded up to 32
     const int m32 = static_cast<int>((m + 31) / 32 * 32);
-    for (int bn : {pair_bn_for(m), 128, 160, 192, 224}) {
-      if (bn > kPairMaxTokens || bn > m32) continue;
+    for (int bn : {pair_bn_for(m), 32, 64, 96, 128, 160, 192, 224}) {
+      if (bn > kPairMaxTokens || bn > m32 || (m >= 256 && bn < 128)) continue;
       for (int ks : {1, 2}) {
         if (k_steps % ks != 0) continue;
         for (int wt : {1, 2}) add(LinearChoice{1, bn, ks, wt, 1});
