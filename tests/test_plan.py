@@ -29,7 +29,9 @@ RULE = [
     ((16, 14336, 4096), dict(pair=0, bn=16, ks=4, whole_tiles=1, ra=1, grid=112)),   # decode
     ((1, 14336, 4096), dict(pair=0, bn=16, ks=4, whole_tiles=1, ra=1, grid=112)),
     ((32, 14336, 4096), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=112)),
-    ((128, 14336, 4096), dict(pair=0, bn=128, ks=2, whole_tiles=1, grid=112)),       # sweep
+    ((128, 14336, 4096), dict(pair=1, bn=128, ks=2, wt=1, grid=112)),                # sweep
+    ((192, 14336, 4096), dict(pair=1, bn=192, ks=2, wt=1)),
+    ((100, 14336, 4096), dict(pair=0, bn=128, ks=2, whole_tiles=1, grid=112)),
     ((128, 4096, 4096), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=128)),
     ((128, 4096, 14336), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=128)),
     ((16, 4096, 14336), dict(pair=0, bn=16, ks=4, whole_tiles=0, grid=148)),        # stream-K
