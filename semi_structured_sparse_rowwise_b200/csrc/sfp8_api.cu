@@ -341,7 +341,7 @@ int producers_for(int stages) { return stages < kPlanProducers ? stages : kPlanP
 // Token count from which the CTA-pair kernel is used; from
 // kPairSmallMinTokens it is used when its tiles keep enough SMs busy.
 constexpr int64_t kPairMinTokens = 512;
-constexpr int64_t kPairSmallMinTokens = 128;
+constexpr int64_t kPairSmallMinTokens = 64;
 // k steps per pipeline stage of the CTA-pair kernel (when k allows).
 constexpr int kPairStepsPerStage = 2;
 // Weight tiles per CTA of the CTA-pair kernel (when there are enough tiles
@@ -390,14 +390,15 @@ LinearChoice default_choice(int64_t m, int64_t n, int64_t k, int num_sms) {
     c.whole = 1;
     return c;
   }
-  // 128..511 tokens: CTA pairs when their tiles keep at least 60 % of the
+  // 64..511 tokens: CTA pairs when their tiles keep at least 60 % of the
   // pairs busy -- the widest token tile first (fewest re-reads of the
   // weight), and at each width two weight tiles per CTA before one (each
   // activation byte feeds twice the MMAs).  Measured in steady state: m=128,
   // 192 on pair tiles of one token tile 13.8 / 15.3 us against 16.9 / 23.5
   // us on the one-CTA kernel (k=4096, n=14336).
   if (m >= kPairSmallMinTokens) {
-    for (int bn = pair_bn_for(m); bn >= 128; bn -= 32) {
+    const int bn0 = pair_bn_for(m);
+    for (int bn = bn0; bn >= (bn0 < 128 ? bn0 : 128); bn -= 32) {
       for (int wt = 2; wt >= 1; --wt) {
         const long long pairs = ((n_tiles + 2 * wt - 1) / (2 * wt)) * ((m + bn - 1) / bn);
         if (pairs * 10 >= 6LL * (num_sms / 2)) {
@@ -432,10 +433,12 @@ LinearChoice default_choice(int64_t m, int64_t n, int64_t k, int num_sms) {
       return c;
     }
   }
-  // Too few tiles even at 16 tokens: split the k range over the SMs.
+  // Too few tiles even at 16 tokens: split the k range over the SMs when
+  // each tile has enough of it (64 k steps or more; measured: m=16, n=4096,
+  // k=14336 is fastest split, k=4096 on 32 whole tiles).
   c.bn = choose_bn(m);
   c.ks = ks_for(c.bn);
-  c.whole = 0;
+  c.whole = k_steps >= 64 ? 0 : 1;
   return c;
 }
 

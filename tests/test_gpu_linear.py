@@ -100,7 +100,7 @@ def test_pair_kernel_deterministic():
 
 
 def test_deterministic_and_counters_reset():
-    m, k, n = 40, 1024, 700            # split-K tiles (grid > tiles)
+    m, k, n = 40, 8192, 700            # split-K tiles (few tiles, 64 k steps each)
     x = synthetic.activation(1, m, k)
     w = synthetic.weight(2, n, k)
     gl = GpuLayer(w, "e4m3")
@@ -120,7 +120,7 @@ def test_deterministic_and_counters_reset():
 
 
 def test_workspace_too_small():
-    m, k, n = 16, 256, 256
+    m, k, n = 16, 8192, 256
     assert S.sfp8_sparse_linear_workspace_bytes(m, n, k) > 16     # split-K shape
     gl = GpuLayer(synthetic.weight(3, n, k), "e4m3")
     aq, sa = S.sfp8_quantize_rowwise(bf16_dev(synthetic.activation(4, m, k)), "e4m3")

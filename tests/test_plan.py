@@ -31,7 +31,11 @@ RULE = [
     ((32, 14336, 4096), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=112)),
     ((128, 14336, 4096), dict(pair=1, bn=128, ks=2, wt=1, grid=112)),                # sweep
     ((192, 14336, 4096), dict(pair=1, bn=192, ks=2, wt=1)),
-    ((100, 14336, 4096), dict(pair=0, bn=128, ks=2, whole_tiles=1, grid=112)),
+    ((100, 14336, 4096), dict(pair=1, bn=128, ks=2, wt=1)),
+    ((64, 14336, 4096), dict(pair=1, bn=64, ks=2, wt=1)),
+    ((96, 14336, 4096), dict(pair=1, bn=96, ks=2, wt=1)),
+    ((32, 14336, 4096), dict(pair=0, bn=32)),
+    ((16, 4096, 4096), dict(pair=0, bn=16, whole_tiles=1, grid=32)),              # short k
     ((128, 4096, 4096), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=128)),
     ((128, 4096, 14336), dict(pair=0, bn=32, ks=4, whole_tiles=1, grid=128)),
     ((16, 4096, 14336), dict(pair=0, bn=16, ks=4, whole_tiles=0, grid=148)),        # stream-K

@@ -63,9 +63,10 @@ def test_noalloc_matches_workspace_entry_point(m, k, n, a_fmt, w_fmt, with_bias)
 
 
 def test_noalloc_rejects_problems_beyond_its_buffer():
-    # 8 weight tiles: too few for the SMs even at 16 tokens per tile, so the
-    # k range is split over 128 CTAs of 128 tokens: 16.8 MB of partial sums
-    m, k, n = 128, 4096, 1024
+    # 8 weight tiles: too few for the SMs even at 16 tokens per tile, and 64
+    # k steps per tile, so the k range is split over 148 CTAs of 128 tokens:
+    # 19.4 MB of partial sums
+    m, k, n = 128, 8192, 1024
     assert S.sfp8_sparse_linear_workspace_bytes(m, n, k) > 8 << 20
     aq = torch.zeros((m, k), dtype=torch.uint8, device="cuda")
     sa = torch.ones((m,), dtype=torch.float32, device="cuda")
