@@ -149,12 +149,12 @@ __global__ void __launch_bounds__(kTwThreads)
   if (lane == 0) red[warp] = amax;
   __syncthreads();
 
-  // ---- publish, arrive, wait (warp 0)
+  // ---- publish and arrive (warp 0, lane 0), then wait or finish the amax
+  __shared__ unsigned int s_prev;
   if (warp == 0) {
     float m = lane < kTwThreads / 32 ? red[lane] : 0.0f;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    unsigned int prev = 0;
     if (lane == 0) {
       if constexpr (kAtomic) {
         if (m > 0.0f) atomicMax(&sync[kTwAtomicAmax], __float_as_uint(m));
@@ -162,39 +162,50 @@ __global__ void __launch_bounds__(kTwThreads)
         partials[blockIdx.x] = m;
       }
       // release: this CTA's partial (or atomic) before its arrival
-      prev = atomic_add_acq_rel_gpu(&sync[kTwArrived], 1u);
+      s_prev = atomic_add_acq_rel_gpu(&sync[kTwArrived], 1u);
     }
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    __syncwarp();   // orders lane 0's acquire before the other lanes' loads
-    int fail = 0;
-    if (prev == gridDim.x - 1) {
-      // Last to arrive: every other CTA's partial is visible (acquire above).
-      float gm = 0.0f;
-      if constexpr (kAtomic) {
-        if (lane == 0) gm = __uint_as_float(atomicExch(&sync[kTwAtomicAmax], 0u));
-      } else {
-        for (unsigned int i = lane; i < gridDim.x; i += 32) gm = fmaxf(gm, __ldcg(&partials[i]));
+  }
+  // orders lane 0's acquire (on the arrival) before every thread's loads below
+  __syncthreads();
+  const bool last = s_prev == gridDim.x - 1;
+  if (last) {
+    // Last to arrive: every other CTA's partial is visible.  The whole CTA
+    // reduces the partials (each thread at most a few loads, issued together).
+    float gm = 0.0f;
+    if constexpr (kAtomic) {
+      if (threadIdx.x == 0) gm = __uint_as_float(atomicExch(&sync[kTwAtomicAmax], 0u));
+    } else {
+      for (unsigned int i = threadIdx.x; i < gridDim.x; i += kTwThreads)
+        gm = fmaxf(gm, __ldcg(&partials[i]));
+    }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-      }
+    for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+    if (lane == 0) red[warp] = gm;
+    __syncthreads();
+    if (warp == 0) {
+      gm = lane < kTwThreads / 32 ? red[lane] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
       if (lane == 0) {
         sync[kTwResult] = __float_as_uint(gm);
         sync[kTwArrived] = 0u;
         store_release_gpu(&sync[kTwGeneration], gen + 1u);
         g_amax = gm;
+        failed = 0;
       }
-    } else if (lane == 0) {
-      const long long t0 = clock64();
-      while (load_acquire_gpu(&sync[kTwGeneration]) == gen) {
-        if (clock64() - t0 > kWaitLimitCycles) {
-          report_device_error(SFP8_DEVICE_TIMEOUT);
-          fail = 1;
-          break;
-        }
-      }
-      if (!fail) g_amax = __uint_as_float(__ldcg(&sync[kTwResult]));
     }
-    if (lane == 0) failed = fail;
+  } else if (threadIdx.x == 0) {
+    int fail = 0;
+    const long long t0 = clock64();
+    while (load_acquire_gpu(&sync[kTwGeneration]) == gen) {
+      if (clock64() - t0 > kWaitLimitCycles) {
+        report_device_error(SFP8_DEVICE_TIMEOUT);
+        fail = 1;
+        break;
+      }
+    }
+    if (!fail) g_amax = __uint_as_float(__ldcg(&sync[kTwResult]));
+    failed = fail;
   }
   __syncthreads();
   if (failed) return;
