@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -543,8 +544,10 @@ struct AlgoEntry {
 };
 std::mutex g_algo_mutex;
 std::vector<AlgoEntry> g_algo_table[kMaxDevices];
+std::atomic<int> g_algo_entries{0};   // entries over all devices: 0 skips the lock
 
 bool lookup_algo(int dev, int64_t m, int64_t n, int64_t k, AlgoEntry* e) {
+  if (g_algo_entries.load(std::memory_order_acquire) == 0) return false;
   std::lock_guard<std::mutex> lock(g_algo_mutex);
   for (const AlgoEntry& a : g_algo_table[dev])
     if (a.m == m && a.n == n && a.k == k) {
@@ -563,8 +566,8 @@ LinearPlan make_plan(int dev, int64_t m, int64_t n, int64_t k, int num_sms) {
 }
 
 template <int BN, int KS, bool RA>
-sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const LinearParams& prm,
-                              int smem_bytes, cudaStream_t st) {
+sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const CUtensorMap& ty,
+                              const LinearParams& prm, int smem_bytes, cudaStream_t st) {
   auto kern = sparse_linear_kernel<BN, KS, RA>;
   const int slot =
       ((BN == 16 ? 0 : BN == 32 ? 1 : BN == 64 ? 2 : BN == 128 ? 3 : 4) * 3 +
@@ -578,7 +581,7 @@ sfp8_status launch_linear_cfg(DeviceInfo* dev, const CUtensorMap& ta, const Line
       dev->smem_attr_set[slot] = true;
     }
   }
-  return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), smem_bytes, st, ta, prm);
+  return launch_dependent(kern, dim3(prm.grid), dim3(kGemmThreads), smem_bytes, st, ta, ty, prm);
 }
 
 // Weight map for the pair kernel with two weight tiles per CTA: the packed
@@ -632,6 +635,22 @@ sfp8_status encode_act_3d(CUtensorMap* map, const void* base, uint64_t m, uint64
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
+}
+
+
+// Output map: y [m, n] bf16 row-major, box 128 columns x box_rows rows.
+sfp8_status encode_y_2d(CUtensorMap* map, void* y, uint64_t m, uint64_t n, uint32_t box_rows) {
+  EncodeTiledFn enc = nullptr;
+  sfp8_status s = get_encoder(&enc);
+  if (s != SFP8_OK) return s;
+  cuuint64_t dims[2] = {n, m};
+  cuuint64_t strides[1] = {n * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileN), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? SFP8_OK : SFP8_ERR_CUDA;
 }
 
@@ -798,29 +817,41 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
   // MMA A operand = weight, B operand = activation.
   prm.idesc = make_idesc_f8f6f4(w_dtype == SFP8_E5M2 ? 1u : 0u, a_dtype == SFP8_E5M2 ? 1u : 0u,
                                 kTileN, static_cast<uint32_t>(pl.bn), true);
+  // y through one TMA store per CTA when each CTA takes one whole tile and
+  // the resident activation's region can stage it (rows of y 16-byte
+  // aligned); otherwise plain stores.  The unused map is a copy of ta.
+  CUtensorMap ty = ta;
+  prm.tma_store = 0;
+  if (pl.ra && pl.whole_tiles && pl.tiles <= pl.grid && n % 8 == 0 && aligned(y, 16) &&
+      static_cast<long long>(pl.bn) * kTileN * 2 <= pl.ra_bytes) {
+    s = encode_y_2d(&ty, y, static_cast<uint64_t>(m), static_cast<uint64_t>(n),
+                    static_cast<uint32_t>(pl.bn));
+    if (s != SFP8_OK) return s;
+    prm.tma_store = 1;
+  }
   const int sm = pl.smem_bytes;
   if (pl.ra) {
     switch (pl.bn * 8 + pl.ks) {
-      case 16 * 8 + 1: return launch_linear_cfg<16, 1, true>(dev, ta, prm, sm, st);
-      case 16 * 8 + 2: return launch_linear_cfg<16, 2, true>(dev, ta, prm, sm, st);
-      case 16 * 8 + 4: return launch_linear_cfg<16, 4, true>(dev, ta, prm, sm, st);
-      case 32 * 8 + 1: return launch_linear_cfg<32, 1, true>(dev, ta, prm, sm, st);
-      case 32 * 8 + 2: return launch_linear_cfg<32, 2, true>(dev, ta, prm, sm, st);
-      case 32 * 8 + 4: return launch_linear_cfg<32, 4, true>(dev, ta, prm, sm, st);
+      case 16 * 8 + 1: return launch_linear_cfg<16, 1, true>(dev, ta, ty, prm, sm, st);
+      case 16 * 8 + 2: return launch_linear_cfg<16, 2, true>(dev, ta, ty, prm, sm, st);
+      case 16 * 8 + 4: return launch_linear_cfg<16, 4, true>(dev, ta, ty, prm, sm, st);
+      case 32 * 8 + 1: return launch_linear_cfg<32, 1, true>(dev, ta, ty, prm, sm, st);
+      case 32 * 8 + 2: return launch_linear_cfg<32, 2, true>(dev, ta, ty, prm, sm, st);
+      case 32 * 8 + 4: return launch_linear_cfg<32, 4, true>(dev, ta, ty, prm, sm, st);
       default: return SFP8_ERR_UNSUPPORTED_SHAPE;   // no such plan is made
     }
   }
   switch (pl.bn * 8 + pl.ks) {
-    case 16 * 8 + 1: return launch_linear_cfg<16, 1, false>(dev, ta, prm, sm, st);
-    case 16 * 8 + 2: return launch_linear_cfg<16, 2, false>(dev, ta, prm, sm, st);
-    case 16 * 8 + 4: return launch_linear_cfg<16, 4, false>(dev, ta, prm, sm, st);
-    case 32 * 8 + 1: return launch_linear_cfg<32, 1, false>(dev, ta, prm, sm, st);
-    case 32 * 8 + 2: return launch_linear_cfg<32, 2, false>(dev, ta, prm, sm, st);
-    case 32 * 8 + 4: return launch_linear_cfg<32, 4, false>(dev, ta, prm, sm, st);
-    case 64 * 8 + 1: return launch_linear_cfg<64, 1, false>(dev, ta, prm, sm, st);
-    case 64 * 8 + 2: return launch_linear_cfg<64, 2, false>(dev, ta, prm, sm, st);
-    case 128 * 8 + 1: return launch_linear_cfg<128, 1, false>(dev, ta, prm, sm, st);
-    case 128 * 8 + 2: return launch_linear_cfg<128, 2, false>(dev, ta, prm, sm, st);
+    case 16 * 8 + 1: return launch_linear_cfg<16, 1, false>(dev, ta, ty, prm, sm, st);
+    case 16 * 8 + 2: return launch_linear_cfg<16, 2, false>(dev, ta, ty, prm, sm, st);
+    case 16 * 8 + 4: return launch_linear_cfg<16, 4, false>(dev, ta, ty, prm, sm, st);
+    case 32 * 8 + 1: return launch_linear_cfg<32, 1, false>(dev, ta, ty, prm, sm, st);
+    case 32 * 8 + 2: return launch_linear_cfg<32, 2, false>(dev, ta, ty, prm, sm, st);
+    case 32 * 8 + 4: return launch_linear_cfg<32, 4, false>(dev, ta, ty, prm, sm, st);
+    case 64 * 8 + 1: return launch_linear_cfg<64, 1, false>(dev, ta, ty, prm, sm, st);
+    case 64 * 8 + 2: return launch_linear_cfg<64, 2, false>(dev, ta, ty, prm, sm, st);
+    case 128 * 8 + 1: return launch_linear_cfg<128, 1, false>(dev, ta, ty, prm, sm, st);
+    case 128 * 8 + 2: return launch_linear_cfg<128, 2, false>(dev, ta, ty, prm, sm, st);
     default: return SFP8_ERR_UNSUPPORTED_SHAPE;   // no such plan is made
   }
 }
@@ -1224,10 +1255,13 @@ sfp8_status sfp8_sparse_linear_set_algo(int64_t m, int64_t n, int64_t k, int alg
   if (algo >= count) return SFP8_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_algo_mutex);
   std::vector<AlgoEntry>& t = g_algo_table[dev->index];
+  const size_t before = t.size();
   t.erase(std::remove_if(t.begin(), t.end(),
                          [&](const AlgoEntry& a) { return a.m == m && a.n == n && a.k == k; }),
           t.end());
   if (algo > 0) t.push_back(AlgoEntry{m, n, k, algo, ch[algo]});
+  g_algo_entries.fetch_add(static_cast<int>(t.size()) - static_cast<int>(before),
+                           std::memory_order_release);
   return SFP8_OK;
 }
 

@@ -113,6 +113,8 @@ struct LinearParams {
   int stages;               // shared-memory pipeline depth (<= kMaxStages)
   int ra_bytes;             // resident activation bytes (BN * k) or 0
   int producers;            // producer warps issuing copies (1..kProducerWarps)
+  int tma_store;            // 1: y through a TMA store from shared memory (one tile per CTA,
+                            // resident activation: its region stages the tile)
   uint32_t idesc;
 };
 
@@ -190,7 +192,8 @@ __device__ __forceinline__ void load_sa(const LinearParams& p, int m0, float (&s
 
 template <int BN, int KS, bool RA>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_a, const LinearParams p) {
+    sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_a,
+                         const __grid_constant__ CUtensorMap tm_y, const LinearParams p) {
   using Cfg = LinearCfg<BN, KS, RA>;
   const int S = p.stages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -492,7 +495,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-        if (whole) {
+        if (whole && p.tma_store) {
+          // stage the bf16 tile [BN tokens][128 rows] in the resident
+          // activation's region, free once the tile's MMAs have completed
+          __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(ra_base);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            stg[(c * 16 + j) * kTileN + n_local] = __float2bfloat16_rn(fmaf(v[j], sa[j] * sw, bv));
+        } else if (whole) {
           store_chunk(p, v, sa, n, mt * BN + c * 16, sw, bv);
         } else if (finish_now) {
           float sum[16];
@@ -515,6 +525,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) part[(c * 16 + j) * kTileN + n_local] = v[j];
+        }
+      }
+      if (whole && p.tma_store) {
+        // one bulk tensor store of the tile; rows past m and columns past n
+        // are clipped by the tensor map
+        fence_proxy_async_smem();
+        named_barrier_sync(1, kEpiThreads);
+        if (warp == kEpiWarp0 && lane == 0) {
+          tma_store_2d(&tm_y, smem_u32(ra_base), nt * kTileN, mt * BN);
+          bulk_commit_group();
+          bulk_wait_group_0();
         }
       }
       tc_fence_before();
