@@ -53,10 +53,10 @@ L2_NOTE = "rotating 8 copies of the compressed weight (8 x 36.7 MB > 126 MB L2)"
 # under profiles/; valid only while the kernel sources hash to `sha1`.
 KERNEL_SOURCES = ("device_common.cuh", "sparse_linear.cuh", "sparse_linear_pair.cuh")
 NCU_TRAFFIC = {
-    ("decode_gate_up_8b", 16): {"sha1": "37c114df6c7baf358acb870bfacac5419466ea07",
-                                "bytes_per_launch": 36888320},
-    ("prefill_8b", 2): {"sha1": "37c114df6c7baf358acb870bfacac5419466ea07",
-                        "bytes_per_launch": 266398464},
+    ("decode_gate_up_8b", 16): {"sha1": "8eae80b6eea5594001909a3d9a075466e4949df6",
+                                "bytes_per_launch": 36889088},
+    ("prefill_8b", 2): {"sha1": "8eae80b6eea5594001909a3d9a075466e4949df6",
+                        "bytes_per_launch": 272412928},
 }
 
 
