@@ -445,10 +445,20 @@ def sfp8_sparse_linear_search(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bia
     return int(best.value), [float(t) for t in times[:count]]
 
 
+# Bumped by every change of the shape-keyed algorithm table made through this
+# binding: workspaces cached for a shape are re-sized when it moves.
+_ALGO_EPOCH = [0]
+
+
+def algo_epoch():
+    return _ALGO_EPOCH[0]
+
+
 def sfp8_sparse_linear_set_algo(m, n, k, algo, device=None):
     with _dev_ctx(device):
         st = load_library().sfp8_sparse_linear_set_algo(m, n, k, algo)
     _check(st, "sfp8_sparse_linear_set_algo")
+    _ALGO_EPOCH[0] += 1
 
 
 def sfp8_sparse_linear_get_algo(m, n, k, device=None):

@@ -48,12 +48,17 @@ class SparseFp8Linear:
 
     def workspace(self, m):
         """The layer's zeroed workspace for m tokens (kept between calls; each
-        call leaves its split-K counters at zero)."""
-        ws = self._ws.get(m)
-        if ws is None:
+        call leaves its split-K counters at zero).  Re-sized after any change
+        of the library's algorithm table (which may pick a split that needs a
+        larger one)."""
+        epoch = B.algo_epoch()
+        hit = self._ws.get(m)
+        if hit is None or hit[0] != epoch:
+            # a fresh zeroed buffer: another split keeps its counters elsewhere
             ws = B.new_quant_workspace(m, self.n, self.k, self.device)
-            self._ws[m] = ws
-        return ws
+            self._ws[m] = (epoch, ws)
+            return ws
+        return hit[1]
 
     def autotune(self, x, reps=10, flush_bytes=256 << 20):
         """Times every work split of the GEMM for x's token count on this
@@ -71,7 +76,6 @@ class SparseFp8Linear:
                                                   self.w_dtype, self.s_w, self.n, self.k,
                                                   bias=self.bias, reps=reps, flush=flush)
         B.sfp8_sparse_linear_set_algo(m, self.n, self.k, best, self.device)
-        self._ws.pop(m, None)       # the workspace size follows the algorithm
         return best, times
 
     def forward(self, x, out=None):
@@ -127,6 +131,7 @@ class HostPipeline:
         self.layer, self.m = layer, m
         self.streams = [torch.cuda.Stream(dev) for _ in range(3)]
         ws = B.new_quant_workspace(m, layer.n, layer.k, dev)
+        self._ws_epoch = B.algo_epoch()
         self.slots = []
         for _ in range(depth):
             self.slots.append(dict(
@@ -153,6 +158,13 @@ class HostPipeline:
         L = self.layer if layer is None else layer
         if (L.n, L.k) != (self.layer.n, self.layer.k):
             raise ValueError("layer shape differs from the pipeline's")
+        if self._ws_epoch != B.algo_epoch():
+            # the algorithm table changed: the forward may need a larger workspace
+            self.synchronize()
+            ws = B.new_quant_workspace(self.m, L.n, L.k, L.device)
+            for s_ in self.slots:
+                s_["ws"] = ws
+            self._ws_epoch = B.algo_epoch()
         # the set is free once its previous forward has read x and its
         # previous copy out has read y
         if sl["used"]:

@@ -132,3 +132,32 @@ def test_layer_autotune_decode_shape():
     finally:
         S.sfp8_sparse_linear_set_algo(m, n, k, 0)
     _status_clean()
+
+
+def test_table_change_resizes_other_layers_workspace():
+    """After one layer's algorithm choice lands in the table, another layer of
+    the same shape (whose workspace was cached under the old choice) still
+    runs: its workspace follows the table."""
+    m, k, n = 16, 8192, 256
+    w = synthetic.weight(12300, n, k)
+    a = S.SparseFp8Linear(bf16_dev(w))
+    b = S.SparseFp8Linear(bf16_dev(w))
+    x = bf16_dev(synthetic.activation(12301, m, k))
+    y0 = b(x).clone()                                   # caches b's workspace
+    count = S.sfp8_sparse_linear_algo_count(m, n, k)
+    # the algorithm with the largest workspace
+    pick = max(range(count), key=lambda i: S.sfp8_sparse_linear_algo_workspace_bytes(m, n, k, i))
+    try:
+        S.sfp8_sparse_linear_set_algo(m, n, k, pick)
+        y1 = b(x)
+        y2 = a(x)
+        torch.cuda.synchronize()
+        assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+        rl = RefLayer(w, "e4m3")
+        rows, aq_r, sa_r = rl.act(synthetic.activation(12301, m, k), "e4m3")
+        y_ref, absdot, scale = rl.linear(aq_r, "e4m3", sa_r)
+        check_output(y1, rows, np.arange(n), y_ref, absdot, scale)
+        check_output(y0, rows, np.arange(n), y_ref, absdot, scale)
+    finally:
+        S.sfp8_sparse_linear_set_algo(m, n, k, 0)
+    _status_clean()
