@@ -28,7 +28,9 @@
  *    as long as they do not share an output or a workspace.
  *  - Deterministic: the same inputs give bit-identical outputs, run to run.
  *  - Empty problems (rows, m or n equal to 0) return SFP8_OK and launch
- *    nothing.
+ *    nothing, except where an entry point states an output for them
+ *    (sfp8_quantize_rowwise with cols == 0 and sfp8_quantize_tensorwise
+ *    with numel == 0 write the guard scale).
  *  - Strides (ld) are in elements.  Row-major everywhere.
  */
 #ifndef SFP8_H_
