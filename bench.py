@@ -484,13 +484,13 @@ def run_ours(args):
             aq2 = torch.empty((m2, k), dtype=torch.uint8, device=dev)
             sa2 = torch.empty((m2,), dtype=torch.float32, device=dev)
             y2 = torch.empty((m2, n), dtype=torch.bfloat16, device=dev)
-            ws2 = S.new_workspace(m2, n, k, dev)
+            ws2 = S.new_quant_workspace(m2, n, k, dev)
 
             def step2(j, x2=x2, aq2=aq2, sa2=sa2, y2=y2, ws2=ws2, m2=m2):
-                S.sfp8_quantize_rowwise(x2, "e4m3", q=aq2, scales=sa2)
+                # the same step as the headline: one library call
                 pk, s = copies[j % WEIGHT_COPIES]
-                S.sfp8_sparse_linear(aq2, "e4m3", sa2, pk, "e4m3", s, n, k, out=y2,
-                                     workspace=ws2)
+                S.sfp8_sparse_linear_quant(x2, "e4m3", pk, "e4m3", s, n, k, out=y2,
+                                           workspace=ws2, a_q=aq2, s_a=sa2)
             for j in range(args.warmup):
                 step2(j)
             g2 = capture(step2, steps)

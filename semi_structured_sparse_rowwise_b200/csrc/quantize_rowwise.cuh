@@ -202,11 +202,13 @@ __device__ __forceinline__ float row_group_max(float v, float* red) {
 }
 
 // Register-resident row quantiser: blockDim = max(TPR, 256) threads,
-// blockDim / TPR rows per block.
+// blockDim / TPR rows per block.  q2, when not null, receives a second copy
+// of the codes (same row stride).
 template <typename T, int kFmt, int TPR, int CHUNKS>
 __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
     quantize_rowwise_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
-                            int64_t ld, uint8_t* __restrict__ q, float* __restrict__ scales) {
+                            int64_t ld, uint8_t* __restrict__ q, float* __restrict__ scales,
+                            uint8_t* __restrict__ q2) {
   grid_dependents_launch();
   grid_dependency_wait();
   using Tr = InputTraits<T>;
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
   if (!row_ok) return;
   if (t == 0) scales[row] = s;
   uint8_t* qr = q + row * cols;
+  uint8_t* qr2 = q2 != nullptr ? q2 + row * cols : nullptr;
 #pragma unroll
   for (int c = 0; c < CHUNKS; ++c) {
     const int64_t vi = static_cast<int64_t>(c) * TPR + t;
@@ -244,6 +247,7 @@ __global__ void __launch_bounds__(TPR > 256 ? TPR : 256)
       uint32_t w[P / 4];
       quantize_vec<kFmt, P>(f, s, r, w);
       store_codes<P>(qr + vi * P, w);
+      if (qr2 != nullptr) store_codes<P>(qr2 + vi * P, w);
     }
   }
 }

@@ -144,11 +144,16 @@ constexpr int64_t kQuantStreamMinRows = 256;
 constexpr int kQuantRingSlots = 24;         // <= kQuantMaxSlots
 constexpr int kQuantSlotsPerConsumer = 1;   // consumers <= kQuantMaxConsumers
 
+// q2 (a second copy of the codes) is honoured by the register-tile path
+// only, which every caller that passes it reaches (fewer than 256 rows of at
+// most 4096 vectors).
 template <typename T, int kFmt>
 sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
-                            float* scales, cudaStream_t st) {
+                            float* scales, cudaStream_t st, void* q2 = nullptr) {
   const T* xp = static_cast<const T*>(x);
   uint8_t* qp = static_cast<uint8_t*>(q);
+  if (q2 != nullptr && (rows >= kQuantStreamMinRows || cols / InputTraits<T>::kPerVec > 4096))
+    return SFP8_ERR_UNSUPPORTED_SHAPE;   // not reached by the callers
   if (cols == 0) {
     const int64_t blocks = (rows + 255) / 256;
     return launch_dependent(quantize_empty_rows_kernel<kFmt>, dim3(static_cast<unsigned>(blocks)),
@@ -192,7 +197,7 @@ sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
     const int64_t per_block = threads / tpr;
     const int64_t blocks = (rows + per_block - 1) / per_block;
     return launch_dependent(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, st, xp,
-                            rows, cols, ld, qp, scales);
+                            rows, cols, ld, qp, scales, static_cast<uint8_t*>(q2));
   };
   if (rows < kQuantStreamMinRows) {
     if (nvec <= 32) return launch(quantize_rowwise_kernel<T, kFmt, 32, 1>, 32);
@@ -214,9 +219,11 @@ sfp8_status launch_quantize(const void* x, int64_t rows, int64_t cols, int64_t l
 
 template <typename T>
 sfp8_status launch_quantize_fmt(const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
-                                sfp8_dtype q_dtype, float* scales, cudaStream_t st) {
-  if (q_dtype == SFP8_E4M3) return launch_quantize<T, SFP8_E4M3>(x, rows, cols, ld, q, scales, st);
-  return launch_quantize<T, SFP8_E5M2>(x, rows, cols, ld, q, scales, st);
+                                sfp8_dtype q_dtype, float* scales, cudaStream_t st,
+                                void* q2 = nullptr) {
+  if (q_dtype == SFP8_E4M3)
+    return launch_quantize<T, SFP8_E4M3>(x, rows, cols, ld, q, scales, st, q2);
+  return launch_quantize<T, SFP8_E5M2>(x, rows, cols, ld, q, scales, st, q2);
 }
 
 // ------------------------------------------------------------------ tensor-wise quantise
@@ -785,11 +792,15 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
                           sfp8_dtype a_dtype, const float* s_a, int64_t m, const void* packed,
                           sfp8_dtype w_dtype, const float* s_w, int64_t n, int64_t k,
                           const void* bias, void* y, float* partials, unsigned int* counters,
-                          cudaStream_t st) {
+                          cudaStream_t st, const void* a_map = nullptr, int64_t a_map_rows = 0) {
   if (pl.pair)
     return launch_pair(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y, st);
+  // The activation map reads a_q's m rows, or a_map_rows rows of a_map (a
+  // copy padded to the token tile: whole rows instead of out-of-range fill).
   CUtensorMap ta;
-  sfp8_status s = encode_act_3d(&ta, a_q, static_cast<uint64_t>(m), static_cast<uint64_t>(k),
+  sfp8_status s = encode_act_3d(&ta, a_map != nullptr ? a_map : a_q,
+                                static_cast<uint64_t>(a_map != nullptr ? a_map_rows : m),
+                                static_cast<uint64_t>(k),
                                 static_cast<uint32_t>(pl.bn),
                                 static_cast<uint32_t>(pl.ra ? pl.k_steps : pl.ks));
   if (s != SFP8_OK) return s;
@@ -856,6 +867,52 @@ sfp8_status launch_linear(DeviceInfo* dev, const LinearPlan& pl, const void* a_q
   }
 }
 
+// Workspace of the one-call forward: the GEMM's split-K scratch, then --
+// with the activation resident and fewer tokens than the tile -- a staging
+// copy of the codes padded to the token tile (256-byte aligned), which the
+// GEMM reads as whole rows (rows past m are never stored, whatever they hold).
+size_t quant_workspace_need(const LinearPlan& pl, int64_t m, int64_t k, bool* pad,
+                            size_t* pad_off) {
+  size_t need = pl.partial_bytes + pl.counter_bytes;
+  *pad = false;
+  *pad_off = 0;
+  if (!pl.pair && pl.ra && m < pl.bn) {
+    *pad = true;
+    *pad_off = (need + 255) & ~static_cast<size_t>(255);
+    need = *pad_off + static_cast<size_t>(pl.bn) * static_cast<size_t>(k);
+  }
+  return need;
+}
+
+// sfp8_quantize_rowwise with an optional second copy of the codes (q2).
+sfp8_status quantize_rowwise_impl(const void* x, sfp8_dtype x_dtype, int64_t rows, int64_t cols,
+                                  int64_t ld_x, void* q, sfp8_dtype q_dtype, float* scales,
+                                  void* stream, void* q2) {
+  if (!is_wide(x_dtype) || !is_fp8(q_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
+  if (rows < 0 || cols < 0 || ld_x < cols) return SFP8_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (rows >= (int64_t(1) << 31) / 8) return SFP8_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return SFP8_OK;
+  if (scales == nullptr || (cols > 0 && (x == nullptr || q == nullptr)))
+    return SFP8_ERR_INVALID_ARG;
+  const int es = elem_size(x_dtype);
+  if (cols > 0 && (!aligned(x, 16) || !aligned(q, 16) || (ld_x * es) % 16 != 0))
+    return SFP8_ERR_MISALIGNED;
+  if (!aligned(scales, 4) || (q2 != nullptr && !aligned(q2, 16))) return SFP8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  sfp8_status s = current_device(&dev);
+  if (s != SFP8_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (x_dtype) {
+    case SFP8_BF16:
+      return launch_quantize_fmt<__nv_bfloat16>(x, rows, cols, ld_x, q, q_dtype, scales, st, q2);
+    case SFP8_F16:
+      return launch_quantize_fmt<__half>(x, rows, cols, ld_x, q, q_dtype, scales, st, q2);
+    default:
+      return launch_quantize_fmt<float>(x, rows, cols, ld_x, q, q_dtype, scales, st, q2);
+  }
+}
+
 }  // namespace
 }  // namespace sfp8
 
@@ -916,29 +973,7 @@ size_t sfp8_compressed_bytes(int64_t n, int64_t k) {
 sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype, int64_t rows, int64_t cols,
                                   int64_t ld_x, void* q, sfp8_dtype q_dtype, float* scales,
                                   void* stream) {
-  if (!is_wide(x_dtype) || !is_fp8(q_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
-  if (rows < 0 || cols < 0 || ld_x < cols) return SFP8_ERR_INVALID_ARG;
-  if (cols % 16 != 0) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (rows >= (int64_t(1) << 31) / 8) return SFP8_ERR_UNSUPPORTED_SHAPE;
-  if (rows == 0) return SFP8_OK;
-  if (scales == nullptr || (cols > 0 && (x == nullptr || q == nullptr)))
-    return SFP8_ERR_INVALID_ARG;
-  const int es = elem_size(x_dtype);
-  if (cols > 0 && (!aligned(x, 16) || !aligned(q, 16) || (ld_x * es) % 16 != 0))
-    return SFP8_ERR_MISALIGNED;
-  if (!aligned(scales, 4)) return SFP8_ERR_MISALIGNED;
-  DeviceInfo* dev = nullptr;
-  sfp8_status s = current_device(&dev);
-  if (s != SFP8_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (x_dtype) {
-    case SFP8_BF16:
-      return launch_quantize_fmt<__nv_bfloat16>(x, rows, cols, ld_x, q, q_dtype, scales, st);
-    case SFP8_F16:
-      return launch_quantize_fmt<__half>(x, rows, cols, ld_x, q, q_dtype, scales, st);
-    default:
-      return launch_quantize_fmt<float>(x, rows, cols, ld_x, q, q_dtype, scales, st);
-  }
+  return quantize_rowwise_impl(x, x_dtype, rows, cols, ld_x, q, q_dtype, scales, stream, nullptr);
 }
 
 size_t sfp8_quantize_tensorwise_workspace_bytes(sfp8_amax_mode mode) {
@@ -1360,7 +1395,9 @@ size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k)
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return 0;
   const LinearPlan pl = make_plan(dev, m, n, k, sms);
-  return pl.partial_bytes + pl.counter_bytes;
+  bool pad = false;
+  size_t pad_off = 0;
+  return quant_workspace_need(pl, m, k, &pad, &pad_off);
 }
 
 sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
@@ -1385,7 +1422,9 @@ sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t 
     if (m == 0) return SFP8_OK;
     return sfp8_quantize_rowwise(x, x_dtype, m, k, ld_x, a_q, a_dtype, s_a, stream);
   }
-  const size_t need = pl.partial_bytes + pl.counter_bytes;
+  bool pad = false;
+  size_t pad_off = 0;
+  const size_t need = quant_workspace_need(pl, m, k, &pad, &pad_off);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
   if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -1393,10 +1432,11 @@ sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t 
   unsigned int* counters = pl.counter_bytes > 0
                                ? reinterpret_cast<unsigned int*>(ws + pl.partial_bytes)
                                : nullptr;
-  s = sfp8_quantize_rowwise(x, x_dtype, m, k, ld_x, a_q, a_dtype, s_a, stream);
+  uint8_t* staged = pad ? ws + pad_off : nullptr;
+  s = quantize_rowwise_impl(x, x_dtype, m, k, ld_x, a_q, a_dtype, s_a, stream, staged);
   if (s != SFP8_OK) return s;
   return launch_linear(dev, pl, a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
-                       partials, counters, st);
+                       partials, counters, st, staged, pad ? pl.bn : 0);
 }
 
 sfp8_status sfp8_selftest_timeout(void* stream) {
@@ -1426,7 +1466,9 @@ sfp8_status sfp8_sparse_linear_quant_host(const void* x_host, void* x_dev, sfp8_
     return SFP8_ERR_INVALID_ARG;
   if (!aligned(x_dev, 16)) return SFP8_ERR_MISALIGNED;
   if (!empty) {
-    const size_t need = pl.partial_bytes + pl.counter_bytes;
+    bool pad = false;
+    size_t pad_off = 0;
+    const size_t need = quant_workspace_need(pl, m, k, &pad, &pad_off);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return SFP8_ERR_WORKSPACE;
     if (workspace != nullptr && !aligned(workspace, 16)) return SFP8_ERR_MISALIGNED;
   }
