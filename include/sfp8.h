@@ -354,8 +354,11 @@ sfp8_status sfp8_sparse_linear_set_algo(int64_t m, int64_t n, int64_t k, int alg
 int sfp8_sparse_linear_get_algo(int64_t m, int64_t n, int64_t k);
 
 /*
- * Workspace for sfp8_sparse_linear_quant (the same as sfp8_sparse_linear's
- * for these sizes).
+ * Workspace for sfp8_sparse_linear_quant: sfp8_sparse_linear's for these
+ * sizes, plus, when the GEMM keeps the activation resident and m is below its
+ * token tile (decode with fewer than 16 tokens), a staging area of tile-high
+ * codes that the quantiser writes besides a_q and the GEMM reads as whole
+ * rows.
  */
 size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
