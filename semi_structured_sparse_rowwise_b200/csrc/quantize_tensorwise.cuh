@@ -18,16 +18,16 @@
 // co-resident); CTA b owns a contiguous run of tiles (kTwThreads * kTwUnroll
 // 16-byte vectors each).  Sweep 1 reads the run front to back, kTwBatch
 // tiles per step, folding |x| into a CTA maximum and keeping the last
-// step's tiles in registers.  The CTA then
-// publishes its maximum (a partials slot, or an atomic max on the float's
-// bits -- |x| >= 0, so the unsigned order of the bits is the float order)
-// and arrives on a grid barrier in the workspace; the last CTA to arrive
-// computes the global amax, clears what must start at zero for the next call
-// and opens the barrier by bumping a generation word.  Sweep 2 converts the
-// kept tiles from registers, then the rest of the run back to front, so that
-// the most recently read tiles -- the ones most likely still in L2 -- are
-// re-read first.  The barrier wait is bounded (kWaitLimitCycles); on expiry
-// the CTA records SFP8_DEVICE_TIMEOUT and converts nothing.
+// step's tiles in registers.  The CTA then publishes its maximum (a partials
+// slot, or an atomic max on the float's bits -- |x| >= 0, so the unsigned
+// order of the bits is the float order) and arrives on a grid barrier in the
+// workspace.  The last CTA to arrive computes the global amax (all its
+// threads reduce the partials), clears what must start at zero for the next
+// call and opens the barrier by bumping a generation word.  Sweep 2 converts
+// the kept tiles from registers, then the rest of the run back to front, so
+// that the most recently read tiles -- the ones most likely still in L2 --
+// are re-read first.  The barrier wait is bounded (kWaitLimitCycles); on
+// expiry the CTA records SFP8_DEVICE_TIMEOUT and converts nothing.
 #pragma once
 
 #include "quantize_rowwise.cuh"
