@@ -114,12 +114,14 @@ def test_zero_outputs_still_quantises():
     assert torch.equal(aq, aq2) and torch.equal(sa.view(torch.int32), sa2.view(torch.int32))
 
 
+@pytest.mark.parametrize("m", [3, 16])
 @pytest.mark.parametrize("pinned", [True, False])
-def test_host_path_matches_device_path(pinned):
+def test_host_path_matches_device_path(pinned, m):
     """sfp8_sparse_linear_quant_host (copy in, quantise, linear, copy out in
     one call) gives the device path's bits, from page-locked or pageable host
-    buffers, on repeated calls."""
-    m, k, n = 16, 1024, 700
+    buffers, on repeated calls; m=3 goes through the tile-high staging of the
+    codes."""
+    k, n = 1024, 700
     x = synthetic.activation(8100, m, k, dist="student_t3")
     w = synthetic.weight(8101, n, k)
     b = synthetic.bias(8102, n)
