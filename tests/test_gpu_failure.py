@@ -14,7 +14,7 @@ import torch
 
 import semi_structured_sparse_rowwise_b200 as S
 from semi_structured_sparse_rowwise_b200 import synthetic
-from gpu_pipeline import GpuLayer, RefLayer, bf16_dev, check_output, ensure_library, requires_gpu
+from gpu_pipeline import GpuLayer, RefLayer, check_output, ensure_library, requires_gpu
 
 pytestmark = [pytest.mark.gpu, requires_gpu]
 

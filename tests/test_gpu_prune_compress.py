@@ -8,8 +8,8 @@ import torch
 import oracle
 import semi_structured_sparse_rowwise_b200 as S
 from semi_structured_sparse_rowwise_b200 import synthetic
-from gpu_pipeline import (GpuLayer, RefLayer, bf16_bits_of, bf16_dev, check_weight_prep,
-                          ensure_library, f32_to_bits16, requires_gpu, sample_indices)
+from gpu_pipeline import (GpuLayer, RefLayer, check_weight_prep, ensure_library, requires_gpu,
+                          sample_indices)
 
 pytestmark = [pytest.mark.gpu, requires_gpu]
 

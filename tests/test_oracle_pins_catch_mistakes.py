@@ -13,7 +13,6 @@ import numpy as np
 
 import oracle
 from oracle import E4M3
-from oracle import fp8 as fp8_mod
 from oracle import prune as prune_mod
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
