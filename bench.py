@@ -236,9 +236,14 @@ def oracle_step_rate(m, seconds=10.0, n_sample=512):
     frac = n_sample / N_DIM
     step_time = dt / reps / frac
     rate = compressed_weight_bytes(N_DIM, K_DIM) / step_time / 1e9
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except Exception:
+        affinity = None
     note = ("oracle (numpy fp64) quantise of the %dx%d activation + linear for %d of %d "
-            "output columns, %d repetitions in %.1f s, scaled to the full N"
-            % (m, K_DIM, n_sample, N_DIM, reps, dt))
+            "output columns, %d repetitions in %.1f s, scaled to the full N; %d BLAS threads, "
+            "os.cpu_count() %s, affinity %s"
+            % (m, K_DIM, n_sample, N_DIM, reps, dt, cores, os.cpu_count(), affinity))
     return rate, cores, note, step_time
 
 
