@@ -31,6 +31,7 @@ class SparseFp8Linear:
             self.packed = B.sfp8_compress_24(w_q, w_dtype)
         self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
         self._ws = {}
+        self._act = {}
         self._host = {}
 
     @classmethod
@@ -43,6 +44,7 @@ class SparseFp8Linear:
         self.packed, self.s_w = packed, s_w
         self.bias = None if bias is None else bias.to(torch.bfloat16).contiguous()
         self._ws = {}
+        self._act = {}
         self._host = {}
         return self
 
@@ -82,22 +84,36 @@ class SparseFp8Linear:
         """x [m, k] bf16/f16/f32 on the layer's device -> y [m, n] bf16.
 
         One library call (sfp8_sparse_linear_quant): the quantiser, then the
-        GEMM as its programmatic dependent."""
+        GEMM as its programmatic dependent.  The quantised activation, its
+        scales and the workspace are kept per token count, so one forward of
+        a layer per token count may be in flight at a time (calls on one
+        stream are ordered)."""
+        m = x.shape[0]
+        a_q, s_a = self._act_buffers(m)
         y, _, _ = B.sfp8_sparse_linear_quant(x, self.a_dtype, self.packed, self.w_dtype,
                                              self.s_w, self.n, self.k, bias=self.bias, out=out,
-                                             workspace=self.workspace(x.shape[0]))
+                                             workspace=self.workspace(m), a_q=a_q, s_a=s_a)
         return y
 
     __call__ = forward
 
+    def _act_buffers(self, m):
+        """The quantised activation [m, k] and its scales [m] (kept per m)."""
+        b = self._act.get(m)
+        if b is None:
+            b = (torch.empty((m, self.k), dtype=torch.uint8, device=self.device),
+                 torch.empty((m,), dtype=torch.float32, device=self.device))
+            self._act[m] = b
+        return b
+
     def _host_buffers(self, m, x_dtype):
-        """Device staging buffers of the host path for m tokens (kept)."""
+        """Device buffers of the host path for m tokens (kept): staging x, the
+        quantised activation and its scales, staging y."""
         key = (m, x_dtype)
         b = self._host.get(key)
         if b is None:
-            b = (torch.empty((m, self.k), dtype=x_dtype, device=self.device),
-                 torch.empty((m, self.k), dtype=torch.uint8, device=self.device),
-                 torch.empty((m,), dtype=torch.float32, device=self.device),
+            a_q, s_a = self._act_buffers(m)
+            b = (torch.empty((m, self.k), dtype=x_dtype, device=self.device), a_q, s_a,
                  torch.empty((m, self.n), dtype=torch.bfloat16, device=self.device))
             self._host[key] = b
         return b
