@@ -32,6 +32,17 @@
  *    (sfp8_quantize_rowwise with cols == 0 and sfp8_quantize_tensorwise
  *    with numel == 0 write the guard scale).
  *  - Strides (ld) are in elements.  Row-major everywhere.
+ *
+ * Typical use (one layer, W [n, k] bf16, k % 128 == 0):
+ *   once:     packed <- sfp8_compressed_bytes(n, k) bytes, s_w <- n floats;
+ *             sfp8_prepare_weight_24(W, SFP8_BF16, n, k, k, SFP8_E4M3, packed, s_w, st);
+ *             ws <- sfp8_sparse_linear_quant_workspace_bytes(m, n, k) bytes, zeroed
+ *             (sfp8_workspace_clear);
+ *   per call: sfp8_sparse_linear_quant(x, SFP8_BF16, k, SFP8_E4M3, a_q, s_a, m,
+ *                                      packed, SFP8_E4M3, s_w, n, k, bias, y,
+ *                                      ws, ws_bytes, st);
+ *   optional: sfp8_sparse_linear_search + sfp8_sparse_linear_set_algo to pick
+ *             the work split for a token count (before sizing ws).
  */
 #ifndef SFP8_H_
 #define SFP8_H_
