@@ -12,6 +12,7 @@ import ml_dtypes
 import numpy as np
 
 import oracle
+import quotient_pin
 from oracle import E4M3
 from oracle import prune as prune_mod
 
@@ -165,3 +166,62 @@ def test_tensorwise_mistakes_are_caught():
     assert _global_amax_pin(oracle.quantize_tensorwise)
     assert not _global_amax_pin(per_block_amax)
     assert not _global_amax_pin(last_block_amax)
+
+
+def _quotient_pins(quantize_rowwise, quantize_tensorwise):
+    """The two quotient pins: the hand-worked inexact-scale row, and codes equal
+    to RN_sat(RN32(x / s)) computed without the oracle on inexact-scale rows."""
+    row = GOLDEN["inexact_scale_row_e4m3"]
+    x = np.array(row["x_bf16_values"], np.float32)[None, :]
+    q, _ = quantize_rowwise(x, E4M3)
+    golden_ok = [int(c) for c in q[0]] == [int(c, 16) for c in row["codes"]]
+    rows = quotient_pin.inexact_scale_rows(23, E4M3)[:128]
+    q, s = quantize_rowwise(rows, E4M3)
+    rowwise_ok = np.array_equal(q, quotient_pin.codes(rows, s[:, None], E4M3))
+    tensor_ok = True
+    for x1 in rows[::8]:
+        q1, s1 = quantize_tensorwise(x1, E4M3)
+        tensor_ok &= np.array_equal(q1, quotient_pin.codes(x1, s1, E4M3))
+    return golden_ok, rowwise_ok, tensor_ok
+
+
+def test_multiply_by_reciprocal_is_caught():
+    """x * RN32(1/s) instead of the correctly rounded x / s, in either quantiser."""
+    def rowwise_recip(x32, fmt):
+        x32 = np.asarray(x32, np.float32)
+        amax = np.max(np.abs(x32), axis=1).astype(np.float32)
+        s = (np.maximum(amax, oracle.GUARD_AMAX) / np.float32(oracle.fp8_max(fmt))).astype(np.float32)
+        r = (np.float32(1.0) / s).astype(np.float32)
+        return oracle.encode_rne_sat((x32 * r[:, None]).astype(np.float32), fmt), s
+
+    def tensorwise_recip(x32, fmt):
+        x32 = np.asarray(x32, np.float32)
+        s = np.float32(np.maximum(np.float32(np.max(np.abs(x32))), oracle.GUARD_AMAX)
+                       / np.float32(oracle.fp8_max(fmt)))
+        return oracle.encode_rne_sat((x32 * np.float32(np.float32(1.0) / s)).astype(np.float32), fmt), s
+
+    assert _quotient_pins(oracle.quantize_rowwise, oracle.quantize_tensorwise) == (True, True, True)
+    golden_ok, rowwise_ok, tensor_ok = _quotient_pins(rowwise_recip, tensorwise_recip)
+    assert not golden_ok and not rowwise_ok and not tensor_ok
+
+
+def test_quotient_rounded_straight_from_float64_is_caught():
+    """x / s evaluated in float64 and rounded once to FP8 (no float32 quotient)."""
+    def rowwise_f64(x32, fmt):
+        x32 = np.asarray(x32, np.float32)
+        amax = np.max(np.abs(x32), axis=1).astype(np.float32)
+        s = (np.maximum(amax, oracle.GUARD_AMAX) / np.float32(oracle.fp8_max(fmt))).astype(np.float32)
+        t = x32.astype(np.float64) / s[:, None].astype(np.float64)
+        table = oracle.decode_table(fmt)
+        top = oracle.max_code(fmt)
+        pos = table[: top + 1]
+        a = np.abs(t)
+        hi = np.minimum(np.searchsorted(pos, a), top)
+        lo = np.maximum(hi - 1, 0)
+        d_lo, d_hi = a - pos[lo], pos[hi] - a
+        mag = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+        mag = np.where(a >= pos[top], top, mag)
+        return (mag | (np.signbit(t).astype(np.int64) << 7)).astype(np.uint8), s
+
+    golden_ok, rowwise_ok, _ = _quotient_pins(rowwise_f64, oracle.quantize_tensorwise)
+    assert not golden_ok and not rowwise_ok

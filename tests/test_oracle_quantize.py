@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 
 import oracle
+import quotient_pin
 from oracle import E4M3, E5M2
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
@@ -107,3 +108,35 @@ def test_scale_is_ieee_float32_division(fmt):
     sd = s.astype(np.float64)
     # s is the float32 nearest to the exact quotient
     assert np.all(np.abs(sd - exact) <= np.minimum(np.abs(lo - exact), np.abs(hi - exact)))
+
+
+def test_inexact_scale_hand_worked_row():
+    """A row with an inexact scale where RN32(x/s) sits on an e4m3 midpoint and
+    ties to the even code, while x * RN32(1/s) would round past it (golden
+    file, worked by hand with integer arithmetic)."""
+    row = GOLDEN["inexact_scale_row_e4m3"]
+    bits = np.array([int(b, 16) for b in row["x_bf16_bits"]], dtype=np.uint16)
+    x = oracle.bf16_bits_to_f32(bits)[None, :]
+    q, s = oracle.quantize_rowwise(x, E4M3)
+    assert s.view(np.uint32)[0] == int(row["scale_bits"], 16)
+    assert s[0] == np.float32(row["scale"])
+    assert [int(c) for c in q[0]] == [int(c, 16) for c in row["codes"]]
+    assert np.array_equal(oracle.decode(q[0], E4M3), np.array(row["decoded"]))
+    assert row["codes"] != row["codes_if_multiplied_by_reciprocal"]
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_quotient_is_one_float32_division(fmt):
+    """Codes equal RN_sat(RN32(x / s)) computed without the oracle (float64
+    quotient rounded once to float32, library cast) on 640 rows whose scales
+    are not powers of two, with values placed beside the FP8 midpoints."""
+    x = quotient_pin.inexact_scale_rows(21, fmt)
+    q, s = oracle.quantize_rowwise(x, fmt)
+    s_ind = quotient_pin.scale(np.abs(x).max(axis=1), fmt)
+    assert np.array_equal(s.view(np.uint32), s_ind.view(np.uint32))
+    assert np.array_equal(q, quotient_pin.codes(x, s_ind[:, None], fmt))
+    # the rows do separate the two readings: multiplying by RN32(1/s) moves codes
+    r = (np.float32(1.0) / s_ind).astype(np.float32)
+    t_mul = (x * r[:, None]).astype(np.float32)
+    q_mul = quotient_pin.codes(t_mul, np.float32(1.0), fmt)
+    assert np.count_nonzero(q_mul != q) > 0

@@ -18,6 +18,7 @@ import numpy as np
 import pytest
 
 import oracle
+import quotient_pin
 from oracle import E4M3, E5M2
 
 GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
@@ -83,3 +84,19 @@ def test_zero_tensor_and_empty(fmt):
     assert q[1, 2] == 0x80 and np.count_nonzero(q) == 1
     q0, s0 = oracle.quantize_tensorwise(np.zeros((0,), np.float32), fmt)
     assert q0.size == 0 and s0 == s
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2])
+def test_quotient_is_one_float32_division(fmt):
+    """Each tensor of a family with inexact scales quantises to RN_sat(RN32(x / s))
+    computed without the oracle (float64 quotient rounded once, library cast)."""
+    rows = quotient_pin.inexact_scale_rows(22, fmt)
+    moved = 0
+    for x in rows[::5]:
+        q, s = oracle.quantize_tensorwise(x, fmt)
+        s_ind = quotient_pin.scale(np.abs(x).max(), fmt)
+        assert np.float32(s).view(np.uint32) == s_ind.view(np.uint32)
+        assert np.array_equal(q, quotient_pin.codes(x, s_ind, fmt))
+        t_mul = (x * (np.float32(1.0) / s_ind).astype(np.float32)).astype(np.float32)
+        moved += np.count_nonzero(quotient_pin.codes(t_mul, np.float32(1.0), fmt) != q)
+    assert moved > 0
