@@ -43,6 +43,12 @@
  *                                      ws, ws_bytes, st);
  *   optional: sfp8_sparse_linear_search + sfp8_sparse_linear_set_algo to pick
  *             the work split for a token count (before sizing ws).
+ *
+ * The compressed weight is one packed buffer (kept values and index
+ * metadata interleaved per 128 x 128 tile) rather than separate values and
+ * metadata buffers, so that one copy brings a tile's operands on chip;
+ * sfp8_compressed_values_bytes / sfp8_compressed_meta_bytes give the sizes
+ * of the two parts inside it.
  */
 #ifndef SFP8_H_
 #define SFP8_H_
@@ -176,6 +182,19 @@ sfp8_status sfp8_prune_24(const void* w, sfp8_dtype dtype, int64_t rows,
  */
 int64_t sfp8_padded_rows(int64_t n);
 size_t sfp8_compressed_bytes(int64_t n, int64_t k);
+
+/*
+ * The two parts of that buffer (item 1's converter emits kept values and
+ * index metadata): sfp8_compressed_values_bytes = n_pad * k / 2 bytes of
+ * kept codes and sfp8_compressed_meta_bytes = n_pad * k / 8 bytes of index
+ * nibbles; for k % 128 == 0 their sum is sfp8_compressed_bytes.  The two
+ * parts are not separate buffers: every 128 x 128 tile stores its 8192 value
+ * bytes and then its 2048 metadata bytes (layout below), so that one
+ * contiguous copy brings a tile's operands into shared memory.  Both return
+ * 0 for a negative n or k.
+ */
+size_t sfp8_compressed_values_bytes(int64_t n, int64_t k);
+size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k);
 
 /*
  * 2:4 compression of an FP8 weight (item 1's converter, with item 3's rule
@@ -449,7 +468,12 @@ sfp8_status sfp8_sparse_linear_quant_host(const void* x_host, void* x_dev, sfp8_
  *    exceeds SFP8_NOALLOC_SCRATCH_BYTES are rejected with SFP8_ERR_WORKSPACE
  *    before anything is launched (on a 148-SM B200 this admits any n and k
  *    for m <= 32 and for m >= 512, which need at most 4.8 MB and no scratch;
- *    between them it depends on the work split chosen for n and k).
+ *    between them it depends on the work split chosen for n and k).  That
+ *    statement describes the built-in work split.  An entry stored with
+ *    sfp8_sparse_linear_set_algo for (m, n, k) is used by this call too; its
+ *    scratch is checked against SFP8_NOALLOC_SCRATCH_BYTES in the same way,
+ *    so a stream-K entry may be rejected with SFP8_ERR_WORKSPACE for a shape
+ *    that the built-in split would have admitted.
  *  - The first call on a device looks up the buffer's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    outside any stream capture.
@@ -483,6 +507,15 @@ sfp8_status sfp8_selftest_timeout(void* stream);
  * SFP8_OK otherwise.
  */
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear);
+
+/*
+ * The status of the last device-side work on the current device, without
+ * clearing it: synchronises the device, then returns SFP8_ERR_TIMEOUT when
+ * a bounded wait gave up, SFP8_ERR_DEVICE_CHECK when a device-side check
+ * failed, SFP8_ERR_CUDA when the device cannot be read, SFP8_OK otherwise.
+ * Same word as sfp8_read_device_status (use that one to clear it).
+ */
+sfp8_status sfp8_last_device_status(void);
 
 const char* sfp8_status_string(sfp8_status s);
 int sfp8_layout_version(void);

@@ -9,7 +9,8 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_quantize_rowwise, sfp8_quantize_tensorwise,
                       sfp8_quantize_tensorwise_workspace_bytes, new_tensorwise_workspace,
                       sfp8_prune_24, sfp8_padded_rows,
-                      sfp8_compressed_bytes,
+                      sfp8_compressed_bytes, sfp8_compressed_values_bytes,
+                      sfp8_compressed_meta_bytes, sfp8_last_device_status,
                       sfp8_compress_24, sfp8_decompress_24, sfp8_prepare_weight_24,
                       sfp8_sparse_linear_workspace_bytes, sfp8_workspace_clear,
                       sfp8_sparse_linear, sfp8_sparse_linear_noalloc,
@@ -27,7 +28,8 @@ __all__ = [
     "Sfp8Error", "load_library", "library_path", "new_workspace",
     "sfp8_quantize_rowwise", "sfp8_quantize_tensorwise",
     "sfp8_quantize_tensorwise_workspace_bytes", "new_tensorwise_workspace", "sfp8_prune_24", "sfp8_padded_rows",
-    "sfp8_compressed_bytes",
+    "sfp8_compressed_bytes", "sfp8_compressed_values_bytes", "sfp8_compressed_meta_bytes",
+    "sfp8_last_device_status",
     "sfp8_compress_24", "sfp8_decompress_24", "sfp8_prepare_weight_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
     "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_sparse_linear_quant",

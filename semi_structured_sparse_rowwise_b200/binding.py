@@ -40,6 +40,8 @@ SIGNATURES = {
     "sfp8_prune_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_padded_rows": (_i64, [_i64]),
     "sfp8_compressed_bytes": (_sz, [_i64, _i64]),
+    "sfp8_compressed_values_bytes": (_sz, [_i64, _i64]),
+    "sfp8_compressed_meta_bytes": (_sz, [_i64, _i64]),
     "sfp8_compress_24": (_i32, [_c_void_p, _i32, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_decompress_24": (_i32, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "sfp8_prepare_weight_24": (_i32, [_c_void_p, _i32, _i64, _i64, _i64, _i32, _c_void_p,
@@ -80,6 +82,7 @@ SIGNATURES = {
                                              _i64, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                              _sz, _c_void_p]),
     "sfp8_read_device_status": (_i32, [ctypes.POINTER(ctypes.c_uint32), _i32]),
+    "sfp8_last_device_status": (_i32, []),
     "sfp8_status_string": (ctypes.c_char_p, [_i32]),
     "sfp8_layout_version": (_i32, []),
 }
@@ -303,22 +306,34 @@ def sfp8_workspace_clear(workspace):
     _check(st, "sfp8_workspace_clear")
 
 
-def sfp8_sparse_linear(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bias=None,
-                       out=None, workspace=None):
-    """y [m, n] bf16 = (s_a s_w^T) * (A_q . W_q^T) + bias."""
-    lib = load_library()
-    _require_cuda(a_q, s_a, packed, s_w, bias)
+def _linear_args(a_q, n, k, bias, out):
+    """Shape, dtype and layout checks shared by the sparse linear wrappers,
+    made before anything reaches the library; returns m."""
     if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
         raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
     m = a_q.shape[0]
     if a_q.shape[1] != k:
         raise ValueError("a_q has %d columns, expected k=%d" % (a_q.shape[1], k))
+    if bias is not None and (bias.dtype != torch.bfloat16 or bias.dim() != 1
+                             or bias.shape[0] != n or not bias.is_contiguous()):
+        raise ValueError("bias must be a contiguous bfloat16 vector of n=%d elements" % n)
+    if out is not None and (out.dtype != torch.bfloat16 or tuple(out.shape) != (m, n)
+                            or not out.is_contiguous() or out.device != a_q.device):
+        raise ValueError("out must be a contiguous (m, n) = (%d, %d) bfloat16 tensor on "
+                         "a_q's device" % (m, n))
+    return m
+
+
+def sfp8_sparse_linear(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bias=None,
+                       out=None, workspace=None):
+    """y [m, n] bf16 = (s_a s_w^T) * (A_q . W_q^T) + bias."""
+    lib = load_library()
+    m = _linear_args(a_q, n, k, bias, out)
+    _require_cuda(a_q, s_a, packed, s_w, bias)
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
     if workspace is None:
         workspace = new_workspace(m, n, k, a_q.device)
-    if bias is not None and bias.dtype != torch.bfloat16:
-        raise ValueError("bias must be bfloat16")
     with torch.cuda.device(a_q.device):
         st = lib.sfp8_sparse_linear(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
                                     _ptr(packed), DTYPE[_fp8_name(w_dtype)],
@@ -335,10 +350,8 @@ def sfp8_sparse_linear_noalloc(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k,
     built-in scratch buffer is used instead.  `out` must be given by such a
     caller; only when it is None does this wrapper allocate it with torch."""
     lib = load_library()
+    m = _linear_args(a_q, n, k, bias, out)
     _require_cuda(a_q, s_a, packed, s_w, bias)
-    if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
-        raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
-    m = a_q.shape[0]
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
     with torch.cuda.device(a_q.device):
@@ -402,10 +415,8 @@ def sfp8_sparse_linear_algo(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, algo,
                             out=None, workspace=None):
     """sfp8_sparse_linear with an explicit work split (algorithm index)."""
     lib = load_library()
+    m = _linear_args(a_q, n, k, bias, out)
     _require_cuda(a_q, s_a, packed, s_w, bias)
-    if a_q.dim() != 2 or not a_q.is_contiguous() or a_q.dtype != torch.uint8:
-        raise ValueError("a_q must be a contiguous 2-D uint8 tensor")
-    m = a_q.shape[0]
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=a_q.device)
     if workspace is None:
@@ -425,8 +436,8 @@ def sfp8_sparse_linear_search(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bia
     """Times every work split of the shape (see include/sfp8.h); returns
     (best algorithm, [median microseconds per algorithm])."""
     lib = load_library()
+    m = _linear_args(a_q, n, k, bias, out)
     _require_cuda(a_q, s_a, packed, s_w, bias, flush)
-    m = a_q.shape[0]
     dev = a_q.device
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
@@ -558,6 +569,19 @@ def sfp8_read_device_status(clear=True):
     flags = ctypes.c_uint32(0)
     st = lib.sfp8_read_device_status(ctypes.byref(flags), 1 if clear else 0)
     return st, flags.value
+
+
+def sfp8_last_device_status():
+    """Status of the current device's status word (not cleared); synchronises."""
+    return int(load_library().sfp8_last_device_status())
+
+
+def sfp8_compressed_values_bytes(n, k):
+    return int(load_library().sfp8_compressed_values_bytes(n, k))
+
+
+def sfp8_compressed_meta_bytes(n, k):
+    return int(load_library().sfp8_compressed_meta_bytes(n, k))
 
 
 def sfp8_status_string(status):

@@ -970,6 +970,16 @@ size_t sfp8_compressed_bytes(int64_t n, int64_t k) {
   return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k) * 5 / 8;
 }
 
+size_t sfp8_compressed_values_bytes(int64_t n, int64_t k) {
+  if (n < 0 || k < 0) return 0;
+  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k) / 2;
+}
+
+size_t sfp8_compressed_meta_bytes(int64_t n, int64_t k) {
+  if (n < 0 || k < 0) return 0;
+  return static_cast<size_t>(sfp8_padded_rows(n)) * static_cast<size_t>(k) / 8;
+}
+
 sfp8_status sfp8_quantize_rowwise(const void* x, sfp8_dtype x_dtype, int64_t rows, int64_t cols,
                                   int64_t ld_x, void* q, sfp8_dtype q_dtype, float* scales,
                                   void* stream) {
@@ -1487,6 +1497,11 @@ sfp8_status sfp8_sparse_linear_quant_host(const void* x_host, void* x_dev, sfp8_
     return SFP8_ERR_CUDA;
   }
   return SFP8_OK;
+}
+
+sfp8_status sfp8_last_device_status(void) {
+  uint32_t flags = 0;
+  return sfp8_read_device_status(&flags, 0);
 }
 
 sfp8_status sfp8_read_device_status(uint32_t* flags, int clear) {

@@ -27,8 +27,9 @@ int main(void) {
       (any_fn)sfp8_sparse_linear_get_algo, (any_fn)sfp8_sparse_linear_quant_workspace_bytes,
       (any_fn)sfp8_sparse_linear_quant, (any_fn)sfp8_sparse_linear_quant_host,
       (any_fn)sfp8_sparse_linear_noalloc, (any_fn)sfp8_selftest_timeout,
-      (any_fn)sfp8_read_device_status, (any_fn)sfp8_status_string,
-      (any_fn)sfp8_layout_version};
+      (any_fn)sfp8_read_device_status, (any_fn)sfp8_last_device_status,
+      (any_fn)sfp8_compressed_values_bytes, (any_fn)sfp8_compressed_meta_bytes,
+      (any_fn)sfp8_status_string, (any_fn)sfp8_layout_version};
   for (size_t i = 0; i < sizeof(fns) / sizeof(fns[0]); ++i)
     if (fns[i] == NULL) return 1;
 
@@ -36,6 +37,9 @@ int main(void) {
   if (sfp8_layout_version() != SFP8_LAYOUT_VERSION) return 2;
   if (sfp8_padded_rows(129) != 256 || sfp8_padded_rows(-1) != -1) return 3;
   if (sfp8_compressed_bytes(14336, 4096) != (size_t)36700160) return 4;
+  if (sfp8_compressed_values_bytes(14336, 4096) != (size_t)29360128 ||
+      sfp8_compressed_meta_bytes(14336, 4096) != (size_t)7340032)
+    return 4;
   if (strcmp(sfp8_status_string(SFP8_OK), "ok") != 0) return 5;
   if (strcmp(sfp8_status_string((sfp8_status)99), "unknown status") != 0) return 6;
 

@@ -48,6 +48,11 @@ def test_layout_constants_match(lib):
         assert lib.sfp8_padded_rows(n) == oracle.padded_rows(n)
         for k in (128, 4096, 14336):
             assert lib.sfp8_compressed_bytes(n, k) == oracle.packed_bytes(n, k)
+            npad = oracle.padded_rows(n)
+            assert lib.sfp8_compressed_values_bytes(n, k) == npad * k // 2
+            assert lib.sfp8_compressed_meta_bytes(n, k) == npad * k // 8
+            assert (lib.sfp8_compressed_values_bytes(n, k) + lib.sfp8_compressed_meta_bytes(n, k)
+                    == lib.sfp8_compressed_bytes(n, k))
 
 
 def test_status_strings(lib):
@@ -167,3 +172,39 @@ def test_linear_validation_without_gpu(lib):
     assert qcall(a_dt=0) == 4          # a_q must be FP8
     assert qcall(k=192, ld_x=192) == 2
     assert qcall(m=0) == 0
+
+
+@pytest.mark.parametrize("entry", ["sfp8_sparse_linear", "sfp8_sparse_linear_noalloc",
+                                   "sfp8_sparse_linear_algo"])
+def test_linear_wrappers_reject_bad_arguments_without_gpu(lib, entry):
+    """The binding's sparse linear wrappers check a_q's width, the bias and the
+    output tensor before any call reaches the library (CPU tensors; nothing
+    launches)."""
+    import torch
+    from semi_structured_sparse_rowwise_b200 import binding as B
+    m, n, k = 4, 64, 256
+    a_q = torch.zeros((m, k), dtype=torch.uint8)
+    s = torch.ones((max(m, n),), dtype=torch.float32)
+    packed = torch.zeros((16,), dtype=torch.uint8)
+    extra = (0,) if entry == "sfp8_sparse_linear_algo" else ()
+    f = getattr(B, entry)
+
+    def call(a=a_q, bias=None, out=None):
+        return f(a, "e4m3", s[:m], packed, "e4m3", s[:n], n, k, *extra, bias=bias, out=out)
+
+    with pytest.raises(ValueError, match="columns"):
+        call(a=torch.zeros((m, k - 128), dtype=torch.uint8))          # fewer than k columns
+    with pytest.raises(ValueError, match="uint8"):
+        call(a=torch.zeros((m, 2 * k), dtype=torch.uint8)[:, :k])     # not contiguous
+    with pytest.raises(ValueError, match="bias"):
+        call(bias=torch.zeros((n,), dtype=torch.float32))            # fp32 bias
+    with pytest.raises(ValueError, match="bias"):
+        call(bias=torch.zeros((n - 1,), dtype=torch.bfloat16))       # short bias
+    with pytest.raises(ValueError, match="out"):
+        call(out=torch.zeros((m, n), dtype=torch.float32))           # fp32 out
+    with pytest.raises(ValueError, match="out"):
+        call(out=torch.zeros((m, n + 1), dtype=torch.bfloat16))      # wrong shape
+    with pytest.raises(ValueError, match="out"):
+        call(out=torch.zeros((n, m), dtype=torch.bfloat16).t())      # not contiguous
+    with pytest.raises(ValueError, match="CUDA"):
+        call()                                                       # well-formed, on the CPU
