@@ -3,26 +3,35 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--m 16] [--impl ours|reference]
 
-Workload: the Llama-3.1-8B MLP gate/up projection at decode (K=4096,
-N=14336, M in {1, 4, 16}; the headline line uses M=16), synthetic seeded
-inputs (A ~ N(0,1) bf16, W ~ N(0, 0.02) bf16, magnitude-pruned 2:4, both
-quantised row-wise to e4m3, no bias).
+Headline workload: the Llama-3.1-8B MLP gate/up projection at decode
+(K=4096, N=14336, M in {1, 4, 16}; the headline line uses M=16), synthetic
+seeded inputs (A ~ N(0,1) bf16, W ~ N(0, 0.02) bf16, magnitude-pruned 2:4,
+both quantised row-wise to e4m3, no bias).  The line's `per_workload`
+carries the compute-bound half of the metric from the same run: the four
+Llama-3.1-8B prefill linears at M=8192 (QKV, O, up, down; A with 1 % outlier
+channels), each in dense-equivalent TFLOP/s against 4 x the measured bf16
+peak, burst and sustained.
 
 A step is one forward of the layer: dynamic row-wise FP8 quantisation of the
-activation followed by the sparse FP8 GEMM with its scale epilogue.  The
-weight is prepared once before timing (prune -> quantise -> compress), as the
-layer does at load time; those kernels, and the one-pass preparation that the
-layer uses (sfp8_prepare_weight_24), are timed separately under "offline".
-The metric's unit for this memory-bound shape is GB/s of compressed weight
+activation followed by the sparse FP8 GEMM with its scale epilogue (one
+library call, two kernels).  The weight is prepared once before timing
+(prune -> quantise -> compress), as the layer does at load time; those
+kernels, and the one-pass preparation that the layer uses
+(sfp8_prepare_weight_24), are timed separately under "offline".  The
+metric's unit for the memory-bound decode shape is GB/s of compressed weight
 bytes (kept values + metadata) per step.
 
 Timing: W eager warm-up steps, then exactly K steps captured in one CUDA
-graph and replayed once between CUDA events on the launching stream, with a
-barrier and a device synchronise on both sides; the max over ranks is
-reported.  The K steps rotate over 8 copies of the compressed weight
-(8 x 36.7 MB > the 126 MB L2), so no step finds its weight in L2.  Under
-torchrun every rank runs an independent replica (weak scaling, no data-path
-collective).
+graph; each replay of it is timed between CUDA events on the launching
+stream, with a barrier and a device synchronise on both sides, and the
+reported time is the median over enough replays to fill about a quarter of
+a second (so the clock sampler sees the load), the max over ranks for each.
+The K steps rotate over copies of the compressed weight that together exceed
+the 126 MB L2 (8 x 36.7 MB at decode), so no step finds its weight in L2.
+`e2e` is the same metric through the C-ABI host-buffer call
+(sfp8_sparse_linear_quant_host: copy in from page-locked host memory,
+quantise, linear, copy out).  Under torchrun every rank runs an independent
+replica (weak scaling, no data-path collective).
 
 `--impl reference` times the CPU oracle (test infrastructure) on a bounded
 sample of the same workload instead.
@@ -247,6 +256,42 @@ def oracle_step_rate(m, seconds=10.0, n_sample=512):
     return rate, cores, note, step_time
 
 
+def oracle_prefill_rate(x_bits, w_bits, seconds=3.0, rows=64, n_sample=1024):
+    """Oracle throughput on a bounded sample of one prefill step: quantise
+    `rows` activation rows and compute `n_sample` output columns, repeated for
+    about `seconds`, then extrapolated linearly in M and N to the full shape.
+    Returns (dense-equivalent TFLOP/s, cores, note)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    m, k = x_bits.shape
+    n = w_bits.shape[0]
+    w32 = oracle.bf16_bits_to_f32(w_bits[:n_sample])
+    wq, sw = oracle.quantize_rowwise(oracle.prune_24(w32), "e4m3")
+    vals, nib = oracle.compress_24(wq, "e4m3")
+    x32 = oracle.bf16_bits_to_f32(x_bits[:rows])
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        aq, sa = oracle.quantize_rowwise(x32, "e4m3")
+        oracle.sparse_linear_ref(aq, "e4m3", sa, vals, nib, "e4m3", sw)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    step_time = dt / reps * (m / rows) * (n / n_sample)
+    rate = 2.0 * m * n * k / step_time / 1e12
+    note = ("extrapolated: oracle (numpy fp64) quantise of %d of %d activation rows + linear "
+            "for %d of %d output columns, %d repetitions in %.1f s, scaled linearly to the "
+            "full M and N; %d BLAS threads, os.cpu_count() %s"
+            % (rows, m, n_sample, n, reps, dt, cores, os.cpu_count()))
+    return rate, cores, note
+
+
 def run_reference(args):
     rank, local, world = dist_setup("gloo")
     if rank != 0:
@@ -347,7 +392,7 @@ def run_ours(args):
                               "GB/s": (wbytes_bf16 + compressed_weight_bytes(n, k) + 4 * n)
                               / off["prepare_weight_24"] / 1e6},
     }
-    del packed1, sw1
+    del packed1, sw1, wp, wq, w_dev
 
     # ---- the step's buffers
     n_copies = WEIGHT_COPIES if not prefill else max(
@@ -379,19 +424,28 @@ def run_ours(args):
         step(j)
     torch.cuda.synchronize(dev)
 
-    def capture(fn, count):
+    def capture(fn, count, streams=()):
+        """One CUDA graph of `count` calls of fn(j); `streams` join the capture
+        (fork from and join back to its origin stream)."""
         g = torch.cuda.CUDAGraph()
         s = torch.cuda.Stream(dev)
         s.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(s):
             with torch.cuda.graph(g, stream=s):
+                for x in streams:
+                    x.wait_stream(s)
                 for j in range(count):
                     fn(j)
+                for x in streams:
+                    s.wait_stream(x)
         torch.cuda.current_stream(dev).wait_stream(s)
         torch.cuda.synchronize(dev)
         return g
 
-    def timed(g, sampler=None):
+    def timed_once(g):
+        """One replay of the K-step graph between CUDA events on the launching
+        stream, with a barrier and a device synchronise on both sides; the max
+        over ranks."""
         barrier(world)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -401,15 +455,23 @@ def run_ours(args):
         e1.synchronize()
         torch.cuda.synchronize(dev)
         barrier(world)
-        return e0.elapsed_time(e1)
+        return dist_max(e0.elapsed_time(e1), world, dev)
+
+    def timed(g):
+        """Median over R timed replays (each exactly K steps): R gives about
+        `--timed-seconds` of timed work, at least 30 replays, so that the clock
+        sampler sees the load and one short replay does not decide the
+        number.  Returns (ms per replay, R)."""
+        g.replay()                       # untimed: graph upload
+        torch.cuda.synchronize(dev)
+        first = timed_once(g)
+        replays = args.replays or int(min(2000, max(30, args.timed_seconds * 1e3 / max(first, 1e-3))))
+        return statistics.median([timed_once(g) for _ in range(replays)]), replays
 
     steps = args.steps
     g_step = capture(step, steps)
-    g_step.replay()                      # untimed: graph upload
-    torch.cuda.synchronize(dev)
     with ClockSampler(local) as clk:
-        ms = timed(g_step)
-    ms = dist_max(ms, world, dev)
+        ms, replays = timed(g_step)
     clocks = clk.summary()
     wbytes = compressed_weight_bytes(n, k)
     flops = 2.0 * m * n * k
@@ -421,13 +483,10 @@ def run_ours(args):
     # ---- the dominant kernel alone (sparse GEMM), same rotation
     quantize()
     g_gemm = capture(gemm, steps)
-    g_gemm.replay()
-    torch.cuda.synchronize(dev)
-    ms_gemm = dist_max(timed(g_gemm), world, dev)
+    ms_gemm, _ = timed(g_gemm)
     gemm_us = ms_gemm * 1e3 / steps
     g_q = capture(lambda j: quantize(), steps)
-    g_q.replay()
-    ms_q = dist_max(timed(g_q), world, dev)
+    ms_q, _ = timed(g_q)
     peak, peak_kind = measured_peaks()
     # the dominant kernel of the step: the GEMM
     kernel_us = gemm_us
@@ -441,43 +500,64 @@ def run_ours(args):
     if rec is not None and rec["sha1"] == kernel_source_sha1():
         traffic = rec["bytes_per_launch"]
 
-    # ---- end to end through the layer's host pipeline: every step copies its
-    # activation in from page-locked host memory and its result out to host
-    # memory; copies in, forward and copies out run on three streams with
-    # rotating device buffers (HostPipeline), captured in a CUDA graph of
-    # E2E_CHUNK steps and replayed
-    # one layer per weight copy, rotated like the device step (the weights
-    # together exceed L2)
-    layers = [S.SparseFp8Linear.from_compressed(pk, s_, n, k) for pk, s_ in copies]
+    # ---- end to end through the C-ABI host-buffer call
+    # (sfp8_sparse_linear_quant_host: copy the activation in from page-locked
+    # host memory, quantise, sparse linear, copy the result out, all in one
+    # library call on one stream).  Steps go round-robin to three streams,
+    # each with its own device staging buffers and host output, so one step's
+    # copies overlap the others' kernels; the K steps are captured in one
+    # CUDA graph (forked to the three streams and joined back) and replayed.
     x_host = torch.from_numpy(np.ascontiguousarray(x_bits).view(np.int16)).view(
         torch.bfloat16).pin_memory()
-    y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
-    chunk = min(E2E_CHUNK, steps)
-    reps = max(1, steps // chunk)
-    pipe = S.HostPipeline(layers[0], m, depth=3)
-    g_e2e = pipe.capture([x_host] * chunk, [y_host] * chunk, layers)
-    for _ in range(max(1, args.warmup // chunk)):
-        g_e2e.replay()
+    e2e_streams = [torch.cuda.Stream(dev) for _ in range(3)]
+    sets = [{"x_dev": torch.empty((m, k), dtype=torch.bfloat16, device=dev),
+             "a_q": torch.empty((m, k), dtype=torch.uint8, device=dev),
+             "s_a": torch.empty((m,), dtype=torch.float32, device=dev),
+             "y_dev": torch.empty((m, n), dtype=torch.bfloat16, device=dev),
+             "y_host": torch.empty((m, n), dtype=torch.bfloat16).pin_memory(),
+             "ws": S.new_quant_workspace(m, n, k, dev)} for _ in e2e_streams]
+
+    def host_step(j):
+        sl = sets[j % len(sets)]
+        pk, s_ = copies[j % len(copies)]
+        with torch.cuda.stream(e2e_streams[j % len(e2e_streams)]):
+            S.sfp8_sparse_linear_quant_host(x_host, "e4m3", pk, "e4m3", s_, n, k, sl["x_dev"],
+                                            sl["a_q"], sl["s_a"], sl["y_dev"], sl["y_host"],
+                                            sl["ws"])
+
+    for s_ in e2e_streams:
+        s_.wait_stream(torch.cuda.current_stream(dev))
+    for j in range(args.warmup):
+        host_step(j)
     torch.cuda.synchronize(dev)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        g_e2e.replay()
-    e1.record()
-    e1.synchronize()
-    ms_e2e = dist_max(e0.elapsed_time(e1), world, dev)
-    barrier(world)
-    e2e_steps = reps * chunk
-    e2e_value = (world * flops * e2e_steps / (ms_e2e * 1e-3) / 1e12 if prefill
-                 else world * wbytes * e2e_steps / (ms_e2e * 1e-3) / 1e9)
+    g_e2e = capture(host_step, steps, e2e_streams)
+    ms_e2e, replays_e2e = timed(g_e2e)
+    e2e_value = (world * flops * steps / (ms_e2e * 1e-3) / 1e12 if prefill
+                 else world * wbytes * steps / (ms_e2e * 1e-3) / 1e9)
     e2e = {"value": e2e_value, "unit": "TFLOP/s" if prefill else "GB/s",
            "h2d_bytes_per_step": m * k * 2, "d2h_bytes_per_step": m * n * 2,
-           "ms_per_step": ms_e2e / e2e_steps,
-           "path": "HostPipeline (copy in, SparseFp8Linear forward, copy out on three "
-                   "streams, pinned host buffers, %d rotating weight copies), CUDA graph "
-                   "of %d steps" % (len(layers), chunk)}
+           "ms_per_step": ms_e2e / steps, "replays": replays_e2e,
+           "path": "sfp8_sparse_linear_quant_host (C-ABI: copy in from page-locked host "
+                   "memory, quantise, sparse linear, copy out), steps round-robin on three "
+                   "streams with their own staging buffers, %d rotating weight copies, CUDA "
+                   "graph of %d steps, median of %d replays" % (len(copies), steps, replays_e2e)}
     del g_e2e
+
+    # the layer's own host pipeline (copies on separate streams), for context
+    e2e_pipe = None
+    if not args.no_pipeline:
+        layers = [S.SparseFp8Linear.from_compressed(pk, s_, n, k) for pk, s_ in copies]
+        y_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+        pipe = S.HostPipeline(layers[0], m, depth=3)
+        g_pipe = pipe.capture([x_host] * steps, [y_host] * steps, layers)
+        ms_pipe, replays_pipe = timed(g_pipe)
+        e2e_pipe = {"value": (flops * steps / (ms_pipe * 1e-3) / 1e12 if prefill
+                              else wbytes * steps / (ms_pipe * 1e-3) / 1e9) * world,
+                    "unit": "TFLOP/s" if prefill else "GB/s", "ms_per_step": ms_pipe / steps,
+                    "path": "HostPipeline (copy in, SparseFp8Linear forward, copy out on three "
+                            "streams), CUDA graph of %d steps, median of %d replays"
+                            % (steps, replays_pipe)}
+        del g_pipe, pipe, layers
 
     # ---- the other decode batch sizes (context lines, same method)
     per_m = {}
@@ -499,10 +579,19 @@ def run_ours(args):
             for j in range(args.warmup):
                 step2(j)
             g2 = capture(step2, steps)
-            g2.replay()
-            ms2 = timed(g2)
+            ms2, _ = timed(g2)
             per_m[str(m2)] = {"value": wbytes * steps / (ms2 * 1e-3) / 1e9, "unit": "GB/s",
                               "ms_per_step": ms2 / steps}
+            del g2
+
+    # ---- the prefill linears (M=8192): the compute-bound half of the metric
+    per_workload = {}
+    if not prefill and world == 1 and not args.no_prefill:
+        del g_step, g_gemm, g_q
+        g_step = g_gemm = g_q = None
+        per_workload["prefill_8b"] = [
+            prefill_case(args, S, synthetic, dev, bf16, capture, timed, i, steps)
+            for i in range(4)]
 
     unit = "TFLOP/s" if prefill else "GB/s"
     line = {
@@ -517,6 +606,9 @@ def run_ours(args):
                    "others (%d x %.1f MB + activations and outputs > 126 MB)"
                    % (len(copies), len(copies), wbytes / 1e6),
                    "step": "sfp8_sparse_linear_quant (quantiser + GEMM kernels)",
+                   "timing": "median of %d replays of one CUDA graph of the K steps, each "
+                             "replay between CUDA events with a barrier and a device "
+                             "synchronise on both sides" % replays,
                    "weight_bytes_per_step": wbytes, "seeds": seeds,
                    "parallelism": "replica" if world > 1 else "single"},
         "roofline": {"bound": "tensor" if prefill else "hbm", "achieved": achieved,
@@ -533,12 +625,21 @@ def run_ours(args):
         "clocks": clocks,
         "offline": off_gbs,
     }
+    if e2e_pipe is not None:
+        line["e2e_pipelined"] = e2e_pipe
     if per_m:
         line["per_m"] = per_m
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not prefill:
-        rate, cores, note, _ = oracle_step_rate(m, seconds=args.cpu_seconds)
-        line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": note}
+    if per_workload:
+        line["per_workload"] = per_workload
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if prefill:
+            rate, cores, note = oracle_prefill_rate(x_bits, w_bits, seconds=args.cpu_seconds)
+            line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": cores,
+                                    "kind": "oracle", "sample": note}
+        else:
+            rate, cores, note, _ = oracle_step_rate(m, seconds=args.cpu_seconds)
+            line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": cores,
+                                    "kind": "oracle", "sample": note}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_step, g_gemm, g_q
@@ -546,6 +647,82 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+PREFILL_NAMES = ("qkv", "o", "up", "down")
+
+
+def prefill_case(args, S, synthetic, dev, bf16, capture, timed, shape_index, steps):
+    """One prefill linear (M=8192) on one GPU: the one-call forward (quantiser
+    + GEMM) and the GEMM alone, each a CUDA graph of `steps` launches rotating
+    weight copies beyond L2, timed like the headline; dense-equivalent TFLOP/s
+    against 4 x the measured bf16 peak (burst and sustained), the clocks seen,
+    ncu traffic when a capture of the current kernels exists, and the oracle
+    on a bounded sample, extrapolated."""
+    import torch
+    x_bits, w_bits, _, seeds = synthetic.workload_inputs("prefill_8b", shape_index)
+    m, k = x_bits.shape
+    n = w_bits.shape[0]
+    w_dev = bf16(w_bits)
+    x_dev = bf16(x_bits)
+    packed, sw = S.sfp8_prepare_weight_24(w_dev, "e4m3")
+    del w_dev
+    n_copies = max(2, -(-150 * 2 ** 20 // (packed.numel() + 2 * m * n)))
+    copies = [(packed.clone(), sw.clone()) for _ in range(n_copies)]
+    del packed
+    aq = torch.empty((m, k), dtype=torch.uint8, device=dev)
+    sa = torch.empty((m,), dtype=torch.float32, device=dev)
+    ys = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    ws = S.new_workspace(m, n, k, dev)
+    ws_q = S.new_quant_workspace(m, n, k, dev)
+
+    def step(j):
+        pk, s_ = copies[j % len(copies)]
+        S.sfp8_sparse_linear_quant(x_dev, "e4m3", pk, "e4m3", s_, n, k, out=ys[j % 2],
+                                   workspace=ws_q, a_q=aq, s_a=sa)
+
+    def gemm(j):
+        pk, s_ = copies[j % len(copies)]
+        S.sfp8_sparse_linear(aq, "e4m3", sa, pk, "e4m3", s_, n, k, out=ys[j % 2],
+                             workspace=ws)
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        g = capture(step, steps)
+        ms_step, replays = timed(g)
+        del g
+        g = capture(gemm, steps)
+        ms_gemm, _ = timed(g)
+        del g
+    flops = 2.0 * m * n * k
+    gemm_us = ms_gemm * 1e3 / steps
+    step_us = ms_step * 1e3 / steps
+    tf = flops / (gemm_us * 1e-6) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+    peak_sus, peak_sus_kind = measured_tensor_peak(sustained=True)
+    traffic = None
+    rec = NCU_TRAFFIC.get(("prefill_8b", shape_index))
+    if rec is not None and rec["sha1"] == kernel_source_sha1():
+        traffic = rec["bytes_per_launch"]
+    out = {"shape": PREFILL_NAMES[shape_index], "m": m, "k": k, "n": n, "seeds": seeds,
+           "steps": steps, "replays": replays, "weight_copies": len(copies),
+           "gemm_us": gemm_us, "step_us": step_us, "TFLOP/s": tf,
+           "step_TFLOP/s": flops / (step_us * 1e-6) / 1e12,
+           "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "frac": tf / peak,
+                        "peak_source": peak_kind, "peak_sustained": peak_sus,
+                        "frac_sustained": tf / peak_sus, "unit": "TFLOP/s",
+                        "traffic": traffic, "kernel": "sparse_linear_pair_kernel",
+                        "algorithmic_flop_per_launch": flops},
+           "clocks": clk.summary()}
+    del copies, aq, sa, ys, ws, ws_q, x_dev
+    torch.cuda.empty_cache()
+    if not args.no_cpu_baseline:
+        rate, cores, note = oracle_prefill_rate(x_bits, w_bits, seconds=args.cpu_seconds_prefill)
+        out["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": cores,
+                               "kind": "oracle", "sample": note}
+    return out
 
 
 # ----------------------------------------------------------------- tensor-wise quantiser
@@ -776,6 +953,15 @@ def main():
     ap.add_argument("--all-m", action="store_true", help="also time M=1 and M=4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds-prefill", type=float, default=3.0,
+                    help="oracle seconds per prefill shape in the default run")
+    ap.add_argument("--replays", type=int, default=0,
+                    help="timed replays of each K-step graph (0: about --timed-seconds)")
+    ap.add_argument("--timed-seconds", type=float, default=0.25)
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the four M=8192 prefill shapes of the default run")
+    ap.add_argument("--no-pipeline", action="store_true",
+                    help="skip the layer's HostPipeline end-to-end leg")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
