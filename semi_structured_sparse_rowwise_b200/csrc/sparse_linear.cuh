@@ -30,7 +30,8 @@
 //               is prefetched into L2 at the start.
 //   warp 4      MMA issuer: per k step, copies the metadata block into tensor
 //               memory (tcgen05.cp 128x128b) and issues two 128 x BN x 64
-//               sparse MMAs; frees the stage with tcgen05.commit.
+//               sparse MMAs; frees the stage with tcgen05.commit.  The whole
+//               warp walks the loop and one elected lane issues.
 //   warps 5-8   epilogue: tensor memory -> registers -> scale/bias/bf16 ->
 //               global, or split-K partials to the workspace.
 // Work split, chosen by the host:
@@ -360,7 +361,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the loop (converged, so its operands stay
+    // warp-uniform); one elected lane issues each tcgen05 operation.
+    {
       grid_dependency_wait();   // start the wait limits only once inputs exist
       SegmentWalker walk(p, cta);
       long long tile;
@@ -371,17 +374,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       const uint32_t e_tmem = tmem_base + Cfg::kMetaCol;
       bool ok = true;
-      if (RA) ok = mbar_wait(smem_u32(ra_bar), 0, abort_flag);
+      if (RA) ok = mbar_wait_warp(smem_u32(ra_bar), 0, abort_flag);
+      // Whether the full barrier of `stage` was already seen complete (each
+      // stage tests the next one's right after its first MMA, so that the
+      // barrier's latency overlaps queued tensor work).
+      bool ready = false;
       while (ok && walk.next(tile, u0, u1)) {
-        if (!mbar_wait(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
+        if (!mbar_wait_warp(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int u = u0; u < u1; ++u) {
-          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag)) {
+          if (!ready && !mbar_wait_warp(smem_u32(&full_bar[stage]), phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const int next_stage = stage + 1 == S ? 0 : stage + 1;
+          const uint32_t next_phase = stage + 1 == S ? phase ^ 1u : phase;
           const uint32_t st = smem_u32(stage_base + stage * Cfg::kStageBytes);
 #pragma unroll
           for (int j = 0; j < KS; ++j) {
@@ -394,9 +403,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // k steps j and j + 1 (consecutive tiles, kWTileBytes apart) in one
             // 128 x 256-bit copy
             if constexpr (KS == 1) {
-              tc_cp_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kNoSwizzle));
+              tc_cp_128x128b_w(e_tmem, smem_desc(e_addr, 0, 128, kNoSwizzle));
             } else if (j % 2 == 0) {
-              tc_cp_128x256b(e_tmem + 4 * j, smem_desc(e_addr, kWTileBytes, 128, kNoSwizzle));
+              tc_cp_128x256b_w(e_tmem + 4 * j, smem_desc(e_addr, kWTileBytes, 128, kNoSwizzle));
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -406,18 +415,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               // activation: BN rows x 128 B (128B swizzle, atoms 1024 B apart);
               // each MMA consumes 64 B of every row.
               const uint64_t bdesc = smem_desc(a_addr + 64 * h, 16, 1024, kSwizzle128);
-              mma_sp_f8f6f4(d_tmem, adesc, bdesc, e_tmem + 4 * j + 2 * h, p.idesc,
-                            (u > u0 || j > 0 || h > 0) ? 1u : 0u);
+              mma_sp_f8f6f4_w(d_tmem, adesc, bdesc, e_tmem + 4 * j + 2 * h, p.idesc,
+                              (u > u0 || j > 0 || h > 0) ? 1u : 0u);
+              if (j == 0 && h == 0)
+                ready = mbar_test_warp(smem_u32(&full_bar[next_stage]), next_phase);
             }
           }
-          tc_commit(smem_u32(&empty_bar[stage]));
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          tc_commit_w(smem_u32(&empty_bar[stage]));
+          stage = next_stage;
+          phase = next_phase;
         }
         if (!ok) break;
-        tc_commit(smem_u32(&accf_bar[acc]));
+        tc_commit_w(smem_u32(&accf_bar[acc]));
         if (Cfg::kNumAcc == 2) {
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
@@ -426,9 +435,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       // Every MMA issued must have finished before tensor memory is freed.
-      tc_commit(smem_u32(drain_bar));
+      tc_commit_w(smem_u32(drain_bar));
       volatile int no_abort = 0;
-      mbar_wait(smem_u32(drain_bar), 0, &no_abort);
+      mbar_wait_warp(smem_u32(drain_bar), 0, &no_abort);
     }
   } else {
     // ------------------------------------------------------------ epilogue

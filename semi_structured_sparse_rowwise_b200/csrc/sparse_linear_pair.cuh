@@ -29,7 +29,8 @@
 //               complete on the stage barrier of rank 0, which rank 0 arms
 //               with the byte count of the pair.
 //   warp 4      rank 0: the MMA issuer (metadata copies and MMAs for the pair,
-//               commits multicast to both CTAs' barriers).  Rank 1: only
+//               commits multicast to both CTAs' barriers), the whole warp
+//               walking the loop and one elected lane issuing.  Rank 1: only
 //               allocates and frees tensor memory with rank 0.
 //   warps 5-    epilogue: two warps per tensor-memory lane quadrant (and
 //               weight slot), each taking every other 16-column chunk of the
@@ -243,7 +244,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
     }
   } else if (warp == kPairMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (rank == 0 && lane == 0) {
+    // The whole warp walks the loop (converged, so its operands stay
+    // warp-uniform); one elected lane issues each tcgen05 operation.
+    if (rank == 0) {
       grid_dependency_wait();
       const uint32_t e_tmem = tmem_base + kPairMetaCol;
       int stage = 0;
@@ -252,17 +255,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
       int acc = 0;              // WT = 1: accumulator buffer of this tile
       uint32_t acc_phase = 0;
       bool ok = true;
+      // Whether the full barrier of `stage` was already seen complete: each
+      // stage tests the next one's barrier right after its first MMA, so the
+      // barrier's latency overlaps queued tensor work instead of draining
+      // the pipe between stages.
+      bool ready = false;
       for (int t = pair; ok && t < p.tiles; t += p.pairs) {
         // The accumulator(s) are free once every epilogue warp of the pair
         // has read the tile that last used them.
-        if (!mbar_wait_cluster(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
+        if (!mbar_wait_cluster_warp(smem_u32(&acce_bar[acc]), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         for (int u = 0; u < p.units; ++u) {
-          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag)) {
+          if (!ready && !mbar_wait_warp(smem_u32(&full_bar[stage]), phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const int next_stage = stage + 1 == S ? 0 : stage + 1;
+          const uint32_t next_phase = stage + 1 == S ? phase ^ 1u : phase;
           const uint32_t st = smem_u32(stage_base + stage * SB);
 #pragma unroll
           for (int j = 0; j < KS; ++j) {
@@ -276,28 +286,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
               // metadata of k steps j and j + 1 of this slot (consecutive tiles)
               // in one 128 x 256-bit copy
               if constexpr (KS == 1) {
-                tc_cp_128x128b_pair(e_col, smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
+                tc_cp_128x128b_pair_w(e_col, smem_desc(w_addr + kWValBytes, 0, 128, kNoSwizzle));
               } else if (j % 2 == 0) {
-                tc_cp_128x256b_pair(e_col, smem_desc(w_addr + kWValBytes, kWTileBytes, 128,
-                                                     kNoSwizzle));
+                tc_cp_128x256b_pair_w(e_col, smem_desc(w_addr + kWValBytes, kWTileBytes, 128,
+                                                       kNoSwizzle));
               }
 #pragma unroll
               for (int kh = 0; kh < 2; ++kh) {
                 const uint64_t adesc = smem_desc(w_addr + 32 * kh, 16, 512, kSwizzle64);
                 const uint64_t bdesc = smem_desc(a_addr + 64 * kh, 16, 1024, kSwizzle128);
-                mma_sp_f8f6f4_pair(d_tmem, adesc, bdesc, e_col + 2 * kh, p.idesc,
-                                   (u > 0 || j > 0 || kh > 0) ? 1u : 0u);
+                mma_sp_f8f6f4_pair_w(d_tmem, adesc, bdesc, e_col + 2 * kh, p.idesc,
+                                     (u > 0 || j > 0 || kh > 0) ? 1u : 0u);
+                if (j == 0 && h == 0 && kh == 0)
+                  ready = mbar_test_warp(smem_u32(&full_bar[next_stage]), next_phase);
               }
             }
           }
-          tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
-          if (++stage == S) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          tc_commit_pair_mc_w(smem_u32(&empty_bar[stage]), 0x3);
+          stage = next_stage;
+          phase = next_phase;
         }
         if (!ok) break;
-        tc_commit_pair_mc(smem_u32(&accf_bar[acc]), 0x3);
+        tc_commit_pair_mc_w(smem_u32(&accf_bar[acc]), 0x3);
         if (WT == 1) {
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1u;
@@ -305,9 +315,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
           acc_phase ^= 1u;
         }
       }
-      tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
+      tc_commit_pair_mc_w(smem_u32(drain_bar), 0x1);
       volatile int no_abort = 0;
-      mbar_wait(smem_u32(drain_bar), 0, &no_abort);
+      mbar_wait_warp(smem_u32(drain_bar), 0, &no_abort);
     }
   } else {
     // ------------------------------------------------------------ epilogue
