@@ -689,6 +689,25 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
   return SFP8_OK;
 }
 
+// Token tiles per band of the pair kernel's tile order (pair_tile_coords):
+// keep one operand resident in L2 while the other streams through once.  With
+// half the L2 as the budget: an activation that fits is kept whole (one band:
+// every weight group read once); else a weight that fits is kept (bands of one
+// token tile: the activation read once); else bands of as many token tiles as
+// fit, so the activation is read once and the weight once per band.
+int pair_band(const DeviceInfo* dev, const LinearPlan& pl, int64_t m, int64_t n, int64_t k) {
+  const long long budget = static_cast<long long>(dev->l2_bytes) / 2;
+  const long long a_bytes = static_cast<long long>(m) * k;
+  const long long w_bytes = static_cast<long long>(sfp8_compressed_bytes(n, k));
+  if (a_bytes <= budget) return pl.m_tiles;
+  if (w_bytes <= budget) return 1;
+  const long long per_tile = static_cast<long long>(pl.bn) * k;
+  long long band = budget / (per_tile > 0 ? per_tile : 1);
+  if (band < 1) band = 1;
+  if (band > pl.m_tiles) band = pl.m_tiles;
+  return static_cast<int>(band);
+}
+
 // CTA-pair GEMM: both maps, the co-resident pair count (queried once per
 // device), launch with programmatic stream serialisation.
 template <int KS, int WT>
@@ -755,6 +774,7 @@ sfp8_status launch_pair_cfg(DeviceInfo* dev, const LinearPlan& pl, const void* a
   prm.k_steps = pl.k_steps;
   prm.units = pl.units;
   prm.tiles = static_cast<int>(pl.tiles);
+  prm.band = pair_band(dev, pl, m, n, k);
   prm.pairs = pairs;
   prm.stages = pl.stages;
   prm.stage_bytes = pl.stage_bytes;

@@ -36,8 +36,8 @@
 //               weight slot), each taking every other 16-column chunk of the
 //               accumulator: tensor memory -> registers -> scale/bias/bf16
 //               -> global.
-// Work split: tile t = n-pair * m_tiles + m-tile, pair p takes tiles p,
-// p + pairs, ...  No split-K.  Tensor memory: accumulator b at columns
+// Work split: tile t -> (weight group, token tile) in bands of token tiles
+// (pair_tile_coords), pair p takes tiles p, p + pairs, ...  No split-K.  Tensor memory: accumulator b at columns
 // [224 b, 224 b + BN), metadata of the stage's k steps at 448.
 //
 // Every wait is bounded (device_common.cuh); a timed-out CTA records
@@ -96,12 +96,30 @@ struct PairParams {
   int k_steps;      // k / 128
   int units;        // stages per tile: k_steps / KS
   int tiles;        // n_groups * m_tiles
+  int band;         // token tiles per band of the tile order (see pair_tile_coords)
   int pairs;        // gridDim.x / 2
   int stages;
   int stage_bytes;  // PairCfg<KS>::stage_bytes(bn)
   int producers;
   uint32_t idesc;
 };
+
+// Tile t -> (weight group g, token tile mt).  Tiles run in bands of p.band
+// token tiles; within a band the token tile varies fastest, so the band's
+// activation rows are reused by every weight group while they sit in L2 and
+// each weight group is read once per band.  p.band = m_tiles is one band
+// (every weight group read once); p.band = 1 runs every weight group over one
+// token tile before the next (the weight stays in L2, the activation is read
+// once).  The host picks the band from the operand sizes and the L2 size.
+__device__ __forceinline__ void pair_tile_coords(const PairParams& p, int t, int& g, int& mt) {
+  const int per_band = p.band * p.n_groups;
+  const int b = t / per_band;
+  const int r = t - b * per_band;
+  const int m0 = b * p.band;
+  const int bsize = p.m_tiles - m0 < p.band ? p.m_tiles - m0 : p.band;
+  g = r / bsize;
+  mt = m0 + (r - g * bsize);
+}
 
 __device__ __forceinline__ void load_sa_pair(const PairParams& p, int m0, float (&sa)[16]) {
 #pragma unroll
@@ -178,7 +196,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
       auto full_of = [&](int stage) { return map_to_cta(smem_u32(&full_bar[stage]), 0); };
       auto issue_weight = [&](int stage, int tile, int u) {
         // CTA r holds weight tiles (2 WT) g + WT r + h, h < WT, of group g.
-        const int g = tile / p.m_tiles;
+        int g, mt_unused;
+        pair_tile_coords(p, tile, g, mt_unused);
         const int nt0 = 2 * WT * g + WT * static_cast<int>(rank);
         const uint32_t dst = smem_u32(stage_base + stage * SB);
         // Rank 0 expects both CTAs' bytes of the stage.
@@ -199,7 +218,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
         }
       };
       auto issue_act = [&](int stage, int tile, int u) {
-        const int mt = tile % p.m_tiles;
+        int g_unused, mt;
+        pair_tile_coords(p, tile, g_unused, mt);
         tma_load_3d_pair(smem_u32(stage_base + stage * SB + Cfg::kWBytes), &tm_a, 0,
                          mt * p.bn + static_cast<int>(rank) * (p.bn / 2), u * KS,
                          full_of(stage), pol_a);
@@ -331,8 +351,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<KS, WT>::kTh
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = pair; t < p.tiles; t += p.pairs) {
-      const int g = t / p.m_tiles;
-      const int mt = t % p.m_tiles;
+      int g, mt;
+      pair_tile_coords(p, t, g, mt);
       const int nt = 2 * WT * g + WT * static_cast<int>(rank) + slot;
       const int n = nt * kTileN + q * 32 + lane;
       const float sw = (n < p.n) ? __ldg(p.s_w + n) : 0.0f;
