@@ -10,7 +10,9 @@ both quantised row-wise to e4m3, no bias).  The line's `per_workload`
 carries the compute-bound half of the metric from the same run: the four
 Llama-3.1-8B prefill linears at M=8192 (QKV, O, up, down; A with 1 % outlier
 channels), each in dense-equivalent TFLOP/s against 4 x the measured bf16
-peak, burst and sustained.
+peak, burst and sustained, then the dtype sweep (K=4096, N=14336, M in
+{1, 16, 128, 1024, 8192} x the four e4m3/e5m2 operand pairs) and the
+Llama-3-70B-shaped stress GEMM (16384 x 8192 x 28672).
 
 A step is one forward of the layer: dynamic row-wise FP8 quantisation of the
 activation followed by the sparse FP8 GEMM with its scale epilogue (one
@@ -594,6 +596,15 @@ def run_ours(args):
         per_workload["prefill_8b"] = [
             prefill_case(args, S, synthetic, dev, bf16, capture, timed, i, steps)
             for i in range(4)]
+        if not args.no_sweep:
+            # the other two measured configurations: the dtype sweep (every M and
+            # operand pair) and the 70B-shaped stress GEMM
+            for wl in ("dtype_sweep_8b_up", "stress_70b_mlp"):
+                table, clocks_wl = matrix_cases(args, wl, S, synthetic, dev, bf16)
+                per_workload[wl] = {"table": table, "clocks": clocks_wl,
+                                    "timing": "one CUDA graph of the case's steps, "
+                                              "replayed once after an untimed replay"}
+                torch.cuda.empty_cache()
 
     unit = "TFLOP/s" if prefill else "GB/s"
     line = {
@@ -841,40 +852,36 @@ def run_tensorwise(args):
 
 # ----------------------------------------------------------------- dtype sweep and stress
 
-def run_matrix(args):
+def matrix_cases(args, workload, S, synthetic, dev, bf16, cases=None):
     """Times the one-call forward (quantiser + GEMM) and the GEMM alone for
     every case of the dtype-sweep workload (M in {1, 16, 128, 1024, 8192} x
     the four e4m3/e5m2 operand pairs, K=4096, N=14336, Student-t activations,
     bf16 bias) or for the 70B stress shape (M=16384, K=8192, N=28672, 2 %
     zero rows).  Each case's steps are one CUDA graph rotating enough
-    compressed-weight copies to exceed L2.  Memory-bound cases (M <= 128) are
-    reported in GB/s of compressed weight against the copy peak, the others
-    in dense-equivalent TFLOP/s against 4 x the bf16 peak."""
-    import numpy as np
+    compressed-weight copies to exceed L2, replayed once after an untimed
+    replay.  Memory-bound cases (M <= 128) are reported in GB/s of compressed
+    weight against the copy peak, the others in dense-equivalent TFLOP/s
+    against 4 x the bf16 peak (burst and sustained).  Returns (table, clocks)."""
     import torch
-    rank, local, world = dist_setup("nccl")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    import semi_structured_sparse_rowwise_b200 as S
-    from semi_structured_sparse_rowwise_b200 import synthetic
-    S.load_library()
     hbm_peak, hbm_kind = measured_peaks()
     fl_peak, fl_kind = measured_tensor_peak()
     fl_sus, fl_sus_kind = measured_tensor_peak(sustained=True)
-
-    def bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
-            torch.bfloat16).to(dev)
-
-    if args.workload == "stress_70b_mlp":
-        cases = [(0, "e4m3", "e4m3")]
-    else:
-        cases = [(i, a, w) for i in range(5) for a in ("e4m3", "e5m2") for w in ("e4m3", "e5m2")]
+    if cases is None:
+        if workload == "stress_70b_mlp":
+            cases = [(0, "e4m3", "e4m3")]
+        else:
+            cases = [(i, a, w) for i in range(5) for a in ("e4m3", "e5m2")
+                     for w in ("e4m3", "e5m2")]
     table = []
     w_cache = {}
-    with ClockSampler(local) as clk:
+    inputs = {}
+    with ClockSampler(dev.index) as clk:
         for shape_index, a_fmt, w_fmt in cases:
-            x_bits, w_bits, b_bits, seeds = synthetic.workload_inputs(args.workload, shape_index)
+            if shape_index not in inputs:
+                # the same seeded inputs serve every operand pair of a shape
+                inputs.clear()
+                inputs[shape_index] = synthetic.workload_inputs(workload, shape_index)
+            x_bits, w_bits, b_bits, seeds = inputs[shape_index]
             m, k = x_bits.shape
             n = w_bits.shape[0]
             key = (w_fmt, n, k)
@@ -941,6 +948,28 @@ def run_matrix(args):
                             "step_TFLOP/s": flops / (res["step"] * 1e-6) / 1e12})
             table.append(row)
             del x, ys, aq, sa, ws
+    return table, clk.summary()
+
+
+def run_matrix(args):
+    """The dtype-sweep or stress workload as its own JSON line (matrix_cases)."""
+    import numpy as np
+    import torch
+    rank, local, world = dist_setup("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import semi_structured_sparse_rowwise_b200 as S
+    from semi_structured_sparse_rowwise_b200 import synthetic
+    S.load_library()
+    hbm_peak, hbm_kind = measured_peaks()
+    fl_peak, fl_kind = measured_tensor_peak()
+    fl_sus, fl_sus_kind = measured_tensor_peak(sustained=True)
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    table, clocks = matrix_cases(args, args.workload, S, synthetic, dev, bf16)
     st_, flags = S.sfp8_read_device_status(clear=True)
     if st_ != 0:
         raise RuntimeError("device status %d flags %#x" % (st_, flags))
@@ -952,7 +981,7 @@ def run_matrix(args):
         "config": {"workload": args.workload, "l2": "rotating >= 200 MB of compressed weight"},
         "peaks": {"hbm": [hbm_peak, hbm_kind], "tensor": [fl_peak, fl_kind],
                   "tensor_sustained": [fl_sus, fl_sus_kind]},
-        "table": table, "clocks": clk.summary(),
+        "table": table, "clocks": clocks,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -992,6 +1021,8 @@ def main():
                     "roofline (at least --steps)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the four M=8192 prefill shapes of the default run")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the dtype sweep and the stress shape of the default run")
     ap.add_argument("--no-pipeline", action="store_true",
                     help="skip the layer's HostPipeline end-to-end leg")
     args = ap.parse_args()
