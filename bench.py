@@ -504,6 +504,27 @@ def run_ours(args):
     if rec is not None and rec["sha1"] == kernel_source_sha1():
         traffic = rec["bytes_per_launch"]
 
+    # ---- the fused form of the step (one kernel in which every CTA quantises
+    # the rows itself), timed beside the chained form that the step uses
+    fused = None
+    if not prefill and S.sfp8_sparse_linear_quant_fusable(m, n, k, dev):
+        def step_fused(j):
+            pk, s_ = copies[j % len(copies)]
+            S.sfp8_sparse_linear_quant_fused(x_dev, "e4m3", pk, "e4m3", s_, n, k,
+                                             out=ys[j % len(ys)], workspace=ws_q, a_q=aq, s_a=sa)
+        for j in range(args.warmup):
+            step_fused(j)
+        g_f = capture(step_fused, ksteps)
+        ms_f, _ = timed(g_f)
+        del g_f
+        g_c = capture(step, ksteps)
+        ms_c, _ = timed(g_c)
+        del g_c
+        fused = {"call": "sfp8_sparse_linear_quant_fused", "step_us": ms_f * 1e3 / ksteps,
+                 "chained_step_us": ms_c * 1e3 / ksteps,
+                 "timing": "median of replays of one CUDA graph of %d steps each, same weight "
+                           "rotation" % ksteps}
+
     # ---- end to end through the C-ABI host-buffer call
     # (sfp8_sparse_linear_quant_host: copy the activation in from page-locked
     # host memory, quantise, sparse linear, copy the result out, all in one
@@ -636,6 +657,7 @@ def run_ours(args):
                                        % ksteps,
                      "peak_source": peak_kind},
         "quantize_us_per_launch": ms_q * 1e3 / ksteps,
+        "fused_step": fused,
         "e2e": e2e,
         "gpu_launches": 2 * steps,
         "clocks": clocks,

@@ -396,9 +396,21 @@ size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k)
  * The layer's forward in one call: dynamic row-wise quantisation of the
  * activation (exactly sfp8_quantize_rowwise: page "Add CUTLASS-based
  * row-wise scaled sparse FP8 kernel", items 1 and 4) followed by the sparse
- * linear (exactly sfp8_sparse_linear), both launched on `stream` (the GEMM
- * as a programmatic dependent of the quantiser, so its weight stream starts
- * while the activation is being quantised).
+ * linear (exactly sfp8_sparse_linear), on `stream`.  Two forms, with the same
+ * results bit for bit (a_q, s_a and y):
+ *   chained  the row-wise quantiser, then the GEMM as its programmatic
+ *            dependent (its weight stream starts while the activation is
+ *            being quantised);
+ *   fused    (where sfp8_sparse_linear_quant_fusable(m, n, k): at most 16
+ *            tokens and the activation resident in one token tile) ONE
+ *            kernel: every CTA of the GEMM quantises the m rows itself into
+ *            shared memory while its weight streams in, and the codes and
+ *            scales are also written to a_q and s_a.
+ * sfp8_sparse_linear_quant runs the chained form, the faster of the two on
+ * B200 at every fusable shape measured (1 to 16 tokens, k = 4096,
+ * n = 14336: 8.5-8.9 us against 10.3-15.4 us per step); _chained and _fused
+ * force one form (the fused one returns SFP8_ERR_UNSUPPORTED_SHAPE where it
+ * does not apply).
  *
  *  x       device, [m, ld_x] bf16 / fp16 / fp32 activation, 16-byte aligned,
  *          ld_x >= k, ld_x * element size a multiple of 16.
@@ -408,6 +420,8 @@ size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k)
  *  packed, w_dtype, s_w, n, k, bias, y: as for sfp8_sparse_linear.
  *  workspace  >= sfp8_sparse_linear_quant_workspace_bytes(m, n, k) bytes,
  *          zero before the first call (left zero by every call).
+ *  x must not overlap a_q, s_a or y (the fused kernel reads x in every CTA
+ *  while some CTAs already write a_q and s_a).
  *
  * Returns the first failing status of the two steps (validation of both
  * before anything is launched where the arguments allow).  With n == 0 only
@@ -419,6 +433,26 @@ sfp8_status sfp8_sparse_linear_quant(const void* x, sfp8_dtype x_dtype, int64_t 
                                      const float* s_w, int64_t n, int64_t k,
                                      const void* bias, void* y, void* workspace,
                                      size_t workspace_bytes, void* stream);
+sfp8_status sfp8_sparse_linear_quant_fused(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
+                                           sfp8_dtype a_dtype, void* a_q, float* s_a, int64_t m,
+                                           const void* packed, sfp8_dtype w_dtype,
+                                           const float* s_w, int64_t n, int64_t k,
+                                           const void* bias, void* y, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+sfp8_status sfp8_sparse_linear_quant_chained(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
+                                             sfp8_dtype a_dtype, void* a_q, float* s_a,
+                                             int64_t m, const void* packed, sfp8_dtype w_dtype,
+                                             const float* s_w, int64_t n, int64_t k,
+                                             const void* bias, void* y, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
+/*
+ * 1 when sfp8_sparse_linear_quant_fused accepts (m, n, k) on the current
+ * device (the work split of the shape, from the table or the built-in rule,
+ * keeps a 16-token activation tile resident), else 0 (also for invalid sizes
+ * and without a device).  Host-only query.
+ */
+int sfp8_sparse_linear_quant_fusable(int64_t m, int64_t n, int64_t k);
 
 /*
  * The layer's forward from host memory to host memory in one call: on

@@ -20,7 +20,8 @@ from .binding import (Sfp8Error, load_library, library_path, new_workspace,
                       sfp8_sparse_linear_search, sfp8_sparse_linear_set_algo,
                       sfp8_sparse_linear_get_algo,
                       sfp8_sparse_linear_quant, sfp8_sparse_linear_quant_workspace_bytes,
-                      sfp8_sparse_linear_quant_host,
+                      sfp8_sparse_linear_quant_host, sfp8_sparse_linear_quant_fused,
+                      sfp8_sparse_linear_quant_chained, sfp8_sparse_linear_quant_fusable,
                       new_quant_workspace, sfp8_read_device_status, sfp8_selftest_timeout,
                       sfp8_status_string, sfp8_layout_version)
 from .layer import HostPipeline, SparseFp8Linear
@@ -34,7 +35,8 @@ __all__ = [
     "sfp8_compress_24", "sfp8_decompress_24", "sfp8_prepare_weight_24",
     "sfp8_sparse_linear_workspace_bytes", "sfp8_workspace_clear",
     "sfp8_sparse_linear", "sfp8_sparse_linear_noalloc", "sfp8_sparse_linear_quant",
-    "sfp8_sparse_linear_quant_host",
+    "sfp8_sparse_linear_quant_host", "sfp8_sparse_linear_quant_fused",
+    "sfp8_sparse_linear_quant_chained", "sfp8_sparse_linear_quant_fusable",
     "sfp8_sparse_linear_algo_count", "sfp8_sparse_linear_algo_info",
     "sfp8_sparse_linear_algo_workspace_bytes", "sfp8_sparse_linear_search_workspace_bytes",
     "sfp8_sparse_linear_algo", "sfp8_sparse_linear_search", "sfp8_sparse_linear_set_algo",

@@ -76,6 +76,15 @@ SIGNATURES = {
     "sfp8_sparse_linear_quant": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p, _c_void_p,
                                         _i64, _c_void_p, _i32, _c_void_p, _i64, _i64,
                                         _c_void_p, _c_void_p, _c_void_p, _sz, _c_void_p]),
+    "sfp8_sparse_linear_quant_fused": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p,
+                                              _c_void_p, _i64, _c_void_p, _i32, _c_void_p,
+                                              _i64, _i64, _c_void_p, _c_void_p, _c_void_p,
+                                              _sz, _c_void_p]),
+    "sfp8_sparse_linear_quant_chained": (_i32, [_c_void_p, _i32, _i64, _i32, _c_void_p,
+                                                _c_void_p, _i64, _c_void_p, _i32, _c_void_p,
+                                                _i64, _i64, _c_void_p, _c_void_p, _c_void_p,
+                                                _sz, _c_void_p]),
+    "sfp8_sparse_linear_quant_fusable": (_i32, [_i64, _i64, _i64]),
     "sfp8_selftest_timeout": (_i32, [_c_void_p]),
     "sfp8_sparse_linear_quant_host": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _c_void_p,
                                              _c_void_p, _i64, _c_void_p, _i32, _c_void_p, _i64,
@@ -493,9 +502,39 @@ def sfp8_sparse_linear_quant(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None, 
                              workspace=None, a_q=None, s_a=None):
     """Quantise x [m, k] (bf16/f16/f32, unit column stride) row-wise and apply
     the sparse linear, one library call: returns (y [m, n] bf16,
-    a_q [m, k] uint8, s_a [m] f32)."""
+    a_q [m, k] uint8, s_a [m] f32), by the chained form (quantiser, then
+    the GEMM as its programmatic dependent)."""
+    return _quant_linear("sfp8_sparse_linear_quant", x, a_dtype, packed, w_dtype, s_w, n, k,
+                         bias, out, workspace, a_q, s_a)
+
+
+def sfp8_sparse_linear_quant_fused(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None, out=None,
+                                   workspace=None, a_q=None, s_a=None):
+    """sfp8_sparse_linear_quant in its fused form: one kernel in which every
+    CTA quantises the (at most 16) rows itself.  Raises Sfp8Error
+    (SFP8_ERR_UNSUPPORTED_SHAPE) where the form does not apply."""
+    return _quant_linear("sfp8_sparse_linear_quant_fused", x, a_dtype, packed, w_dtype, s_w, n,
+                         k, bias, out, workspace, a_q, s_a)
+
+
+def sfp8_sparse_linear_quant_chained(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None,
+                                     out=None, workspace=None, a_q=None, s_a=None):
+    """sfp8_sparse_linear_quant in its chained form: the row-wise quantiser,
+    then the GEMM as its programmatic dependent."""
+    return _quant_linear("sfp8_sparse_linear_quant_chained", x, a_dtype, packed, w_dtype, s_w,
+                         n, k, bias, out, workspace, a_q, s_a)
+
+
+def sfp8_sparse_linear_quant_fusable(m, n, k, device=None):
+    """Whether sfp8_sparse_linear_quant_fused accepts (m, n, k) on `device`
+    (host-only query)."""
     lib = load_library()
-    _require_cuda(x, packed, s_w, bias)
+    with _dev_ctx(device):
+        return bool(lib.sfp8_sparse_linear_quant_fusable(m, n, k))
+
+
+def _quant_linear(name, x, a_dtype, packed, w_dtype, s_w, n, k, bias, out, workspace, a_q, s_a):
+    lib = load_library()
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit column stride")
     m = x.shape[0]
@@ -513,16 +552,23 @@ def sfp8_sparse_linear_quant(x, a_dtype, packed, w_dtype, s_w, n, k, bias=None, 
         a_q = torch.empty((m, k), dtype=torch.uint8, device=dev)
     if s_a is None:
         s_a = torch.empty((m,), dtype=torch.float32, device=dev)
+    for t, shape, dtype, what in ((out, (m, n), torch.bfloat16, "out"),
+                                  (a_q, (m, k), torch.uint8, "a_q"),
+                                  (s_a, (m,), torch.float32, "s_a")):
+        if (tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous()
+                or t.device != dev):
+            raise ValueError("%s must be a contiguous %s tensor of shape %s on %s"
+                             % (what, dtype, shape, dev))
+    _require_cuda(x, packed, s_w, bias)
     if workspace is None:
         workspace = new_quant_workspace(m, n, k, dev)
     ld = x.stride(0) if m > 1 else k
     with torch.cuda.device(dev):
-        st = lib.sfp8_sparse_linear_quant(_ptr(x), DTYPE[xd], ld, DTYPE[_fp8_name(a_dtype)],
-                                          _ptr(a_q), _ptr(s_a), m, _ptr(packed),
-                                          DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n, k,
-                                          _ptr(bias), _ptr(out), _ptr(workspace),
-                                          workspace.numel(), _stream(dev))
-    _check(st, "sfp8_sparse_linear_quant")
+        st = getattr(lib, name)(_ptr(x), DTYPE[xd], ld, DTYPE[_fp8_name(a_dtype)], _ptr(a_q),
+                                _ptr(s_a), m, _ptr(packed), DTYPE[_fp8_name(w_dtype)],
+                                _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
+                                workspace.numel(), _stream(dev))
+    _check(st, name)
     return out, a_q, s_a
 
 

@@ -45,6 +45,15 @@
 //                are always added in CTA order, so results are bit-identical
 //                run to run whichever part finishes.
 //
+// Fused activation quantisation (FQ, one token tile of at most 16 tokens):
+// instead of loading codes that the row-wise quantiser wrote, every CTA
+// quantises the activation itself -- warps 5-12 read the m rows of x, reduce
+// each row's amax, and write its codes (the quantiser's own quotient and
+// conversion, so the same bits) straight into the resident activation's
+// swizzled shared-memory tile.  The producers stream the weight meanwhile;
+// the MMA warp waits for the codes.  The codes and scales also go to global
+// memory, each k step of the codes written by one CTA.
+//
 // Every wait is bounded (device_common.cuh): on a timeout the CTA records
 // SFP8_DEVICE_TIMEOUT, lets its copies in flight land, drains its MMAs,
 // frees its tensor memory and returns.
@@ -53,6 +62,7 @@
 #include <cuda_bf16.h>
 
 #include "device_common.cuh"
+#include "quantize_rowwise.cuh"
 
 namespace sfp8 {
 
@@ -67,6 +77,14 @@ constexpr int kEpiWarp0 = kProducerWarps + 1;           // four epilogue warps
 constexpr int kGemmThreads = 32 * (kProducerWarps + 5);
 constexpr int kEpiThreads = 128;
 constexpr int kSmemBudget = 225 * 1024;
+// Fused quantisation: the four epilogue warps and four more quantise.
+constexpr int kFusedQuantWarps = 8;
+constexpr int kFusedQuantThreads = 32 * kFusedQuantWarps;
+constexpr int kFusedMaxTokens = 16;
+constexpr uint32_t kQuantBarrier = 2;   // named barrier of the quantiser warps
+__host__ __device__ constexpr int linear_threads(bool fq) {
+  return kGemmThreads + (fq ? kFusedQuantThreads - kEpiThreads : 0);
+}
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
   int p = 32;
@@ -117,6 +135,13 @@ struct LinearParams {
   int tma_store;            // 1: y through a TMA store from shared memory (one tile per CTA,
                             // resident activation: its region stages the tile)
   uint32_t idesc;
+  // fused quantisation only
+  const void* x;            // activation [m][ld_x], x_dtype
+  long long ld_x;           // row stride of x in elements
+  int x_dtype;              // SFP8_BF16 / SFP8_F16 / SFP8_F32
+  int a_fmt;                // SFP8_E4M3 / SFP8_E5M2
+  uint8_t* a_q_out;         // codes [m][k], written (k step t by CTA t mod grid)
+  float* s_a_out;           // row scales [m], written by CTA 0
 };
 
 // The work of one CTA, one tile segment [u0, u1) (in stages) at a time.  All
@@ -186,15 +211,131 @@ __device__ __forceinline__ void store_chunk(const LinearParams& p, const float (
   }
 }
 
-__device__ __forceinline__ void load_sa(const LinearParams& p, int m0, float (&sa)[16]) {
+template <bool FQ = false>
+__device__ __forceinline__ void load_sa(const LinearParams& p, int m0, float (&sa)[16],
+                                        const float* sa_sm = nullptr) {
 #pragma unroll
-  for (int j = 0; j < 16; ++j) sa[j] = (m0 + j < p.m) ? __ldg(p.s_a + m0 + j) : 0.0f;
+  for (int j = 0; j < 16; ++j) {
+    if constexpr (FQ)
+      sa[j] = (m0 + j < p.m) ? sa_sm[m0 + j] : 0.0f;
+    else
+      sa[j] = (m0 + j < p.m) ? __ldg(p.s_a + m0 + j) : 0.0f;
+  }
 }
 
-template <int BN, int KS, bool RA>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+// Fused quantisation of the m <= 16 rows of x by the kFusedQuantThreads
+// quantiser threads (index qt): per row, amax = max |x| over the row, s =
+// max(amax, 1e-12) / FP8_MAX, codes = satfinite RNE(x / s) -- exactly the
+// arithmetic of quantize_rowwise_kernel.  The rows are spread over all
+// threads (256 / R threads per row, R the row count rounded up to a power of
+// two); x is read twice (amax, then codes; the second read hits L2).  Codes
+// land in `ra` as the tile [k step][16 rows][128 B] with the 128-byte swizzle
+// (16-byte chunk c of row r at chunk c ^ (r mod 8)); rows past m get zero
+// codes.  `red` is shared scratch of kFusedQuantWarps floats.
+template <typename T, int kFmt>
+__device__ __forceinline__ void fused_quantize(const LinearParams& p, int qt, uint8_t* ra,
+                                               float* sa_sm, float* red) {
+  using Tr = InputTraits<T>;
+  constexpr int P = Tr::kPerVec;      // elements per 16-byte vector
+  constexpr int NV = 16 / P;          // vectors per 16 codes
+  constexpr int kTileBytes = kFusedMaxTokens * kStepK;
+  const int rows_p2 = p.m <= 1 ? 1 : p.m <= 2 ? 2 : p.m <= 4 ? 4 : p.m <= 8 ? 8 : 16;
+  const int tpr = kFusedQuantThreads / rows_p2;
+  const int row = qt / tpr;
+  const int sub = qt % tpr;
+  const bool live = row < p.m;
+  const T* xr = static_cast<const T*>(p.x) + static_cast<long long>(live ? row : 0) * p.ld_x;
+  float amax = 0.0f;
+  if (live) {
+    const int nvec = p.k / P;
+#pragma unroll 8
+    for (int v = sub; v < nvec; v += tpr)
+      amax = Tr::abs_max(__ldg(reinterpret_cast<const uint4*>(xr + static_cast<long long>(v) * P)),
+                         amax);
+  }
+  for (int o = (tpr < 32 ? tpr : 32) / 2; o > 0; o >>= 1)
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (tpr > 32) {
+    const int w = qt / 32;
+    if (qt % 32 == 0) red[w] = amax;
+    named_barrier_sync(kQuantBarrier, kFusedQuantThreads);
+    const int wpr = tpr / 32;
+    const int first = (w / wpr) * wpr;
+    float mx = red[first];
+    for (int i = 1; i < wpr; ++i) mx = fmaxf(mx, red[first + i]);
+    amax = mx;
+  }
+  const float s = __fdiv_rn(fmaxf(amax, kGuardAmax), Fp8Out<kFmt>::kMax);
+  const float r = __frcp_rn(s);
+  if (live && sub == 0) {
+    sa_sm[row] = s;
+    if (blockIdx.x == 0) p.s_a_out[row] = s;
+  }
+  const int nchunk = p.k / 16;
+  const int rsw = row % 8;
+  uint8_t* ra_row = ra + (row / 8) * 1024 + rsw * 128;
+  uint8_t* q_row = p.a_q_out + static_cast<long long>(live ? row : 0) * p.k;
+#pragma unroll 4
+  for (int j = sub; j < nchunk; j += tpr) {
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    const int ks = j / 8;
+    if (live) {
+      uint4 v[NV];
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+        v[i] = __ldg(reinterpret_cast<const uint4*>(xr + static_cast<long long>(j) * 16 + i * P));
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        float f[P];
+        Tr::to_float(v[i], f);
+        uint32_t ww[P / 4];
+        quantize_vec<kFmt, P>(f, s, r, ww);
+#pragma unroll
+        for (int t = 0; t < P / 4; ++t) w[i * (P / 4) + t] = ww[t];
+      }
+      out = make_uint4(w[0], w[1], w[2], w[3]);
+      if (ks % p.grid == static_cast<int>(blockIdx.x))
+        *reinterpret_cast<uint4*>(q_row + static_cast<long long>(j) * 16) = out;
+    }
+    *reinterpret_cast<uint4*>(ra_row + ks * kTileBytes + (((j % 8) ^ rsw) * 16)) = out;
+  }
+  // rows that no thread group covers (fewer rows than the tile): zero codes
+  const int rest = (kFusedMaxTokens - rows_p2) * nchunk;
+  for (int idx = qt; idx < rest; idx += kFusedQuantThreads) {
+    const int r2 = rows_p2 + idx / nchunk;
+    const int j = idx % nchunk;
+    *reinterpret_cast<uint4*>(ra + (j / 8) * kTileBytes + (r2 / 8) * 1024 + (r2 % 8) * 128 +
+                              (((j % 8) ^ (r2 % 8)) * 16)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The quantiser threads' part of the fused kernel: codes and scales for the
+// input type and code format of the call, made visible to the MMAs (async
+// proxy) and signalled on `ra_bar`.
+__device__ __forceinline__ void fused_quantize_all(const LinearParams& p, int qt, uint8_t* ra,
+                                                   float* sa_sm, float* red, uint64_t* ra_bar) {
+  const bool e5 = p.a_fmt == SFP8_E5M2;
+  if (p.x_dtype == SFP8_BF16) {
+    if (e5) fused_quantize<__nv_bfloat16, SFP8_E5M2>(p, qt, ra, sa_sm, red);
+    else fused_quantize<__nv_bfloat16, SFP8_E4M3>(p, qt, ra, sa_sm, red);
+  } else if (p.x_dtype == SFP8_F16) {
+    if (e5) fused_quantize<__half, SFP8_E5M2>(p, qt, ra, sa_sm, red);
+    else fused_quantize<__half, SFP8_E4M3>(p, qt, ra, sa_sm, red);
+  } else {
+    if (e5) fused_quantize<float, SFP8_E5M2>(p, qt, ra, sa_sm, red);
+    else fused_quantize<float, SFP8_E4M3>(p, qt, ra, sa_sm, red);
+  }
+  fence_proxy_async_smem();
+  named_barrier_sync(kQuantBarrier, kFusedQuantThreads);
+  if (qt == 0) mbar_arrive(smem_u32(ra_bar));
+}
+
+template <int BN, int KS, bool RA, bool FQ = false>
+__global__ void __launch_bounds__(linear_threads(FQ), 1)
     sparse_linear_kernel(const __grid_constant__ CUtensorMap tm_a,
                          const __grid_constant__ CUtensorMap tm_y, const LinearParams p) {
+  static_assert(!FQ || (RA && BN == kFusedMaxTokens), "fused quantisation: one 16-token tile");
   using Cfg = LinearCfg<BN, KS, RA>;
   const int S = p.stages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -212,6 +353,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * SM + 5);
   uint64_t* drain_bar = bars + 2 * SM + 6;
   uint64_t* ra_bar = bars + 2 * SM + 7;
+  float* sa_sm = reinterpret_cast<float*>(bars + 2 * SM + 8);      // [16] (FQ)
+  float* q_red = reinterpret_cast<float*>(bars + 2 * SM + 16);     // [8] (FQ)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -236,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_a);
+  if (!FQ && warp == 0 && lane == 0) tma_prefetch_desc(&tm_a);
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
     tmem_relinquish();
@@ -313,7 +456,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (RA && pw == P - 1) {
+      if (RA && !FQ && pw == P - 1) {
         // The whole activation slice of this CTA, [k steps][BN rows][128 B],
         // in one copy by the warp that issued the fewest prefetch copies.
         grid_dependency_wait();
@@ -353,7 +496,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           volatile int no_abort = 0;
           mbar_wait(smem_u32(&full_bar[s2]), ph, &no_abort);
         }
-        if (RA && pw == P - 1) {
+        if (RA && !FQ && pw == P - 1) {
           volatile int no_abort = 0;
           mbar_wait(smem_u32(ra_bar), 0, &no_abort);
         }
@@ -439,12 +582,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       volatile int no_abort = 0;
       mbar_wait_warp(smem_u32(drain_bar), 0, &no_abort);
     }
+  } else if (FQ && warp >= kEpiWarp0 + 4) {
+    // ------------------------------------------------------------ quantiser only
+    grid_dependency_wait();
+    fused_quantize_all(p, threadIdx.x - 32 * kEpiWarp0, ra_base, sa_sm, q_red, ra_bar);
   } else {
     // ------------------------------------------------------------ epilogue
     // Each of the four warps owns 32 weight rows (its tensor-memory lane
     // quadrant) and finishes them on its own, split-K fix-up included, so no
     // barrier spans the four warps.
     grid_dependency_wait();
+    if constexpr (FQ)
+      fused_quantize_all(p, threadIdx.x - 32 * kEpiWarp0, ra_base, sa_sm, q_red, ra_bar);
     const int q = warp % 4;
     SegmentWalker walk(p, cta);
     long long tile;
@@ -464,7 +613,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const float sw = (n < p.n) ? __ldg(p.s_w + n) : 0.0f;
       const float bv = (p.bias != nullptr && n < p.n) ? __bfloat162float(p.bias[n]) : 0.0f;
       float sa0[16];
-      load_sa(p, mt * BN, sa0);
+      load_sa<FQ>(p, mt * BN, sa0, sa_sm);
       int c_first = cta, c_last = cta;
       unsigned int parts = 1;
       unsigned int* counter = p.counters + tile * 4 + q;
@@ -498,7 +647,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) sa[j] = sa0[j];
         } else {
-          load_sa(p, mt * BN + c * 16, sa);
+          load_sa<FQ>(p, mt * BN + c * 16, sa, sa_sm);
         }
         tmem_ld_wait();
         float v[16];
@@ -572,7 +721,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < BN / 16; ++c) {
             float sa[16];
-            load_sa(p, mt * BN + c * 16, sa);
+            load_sa<FQ>(p, mt * BN + c * 16, sa, sa_sm);
             float v[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.0f;

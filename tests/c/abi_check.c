@@ -26,6 +26,8 @@ int main(void) {
       (any_fn)sfp8_sparse_linear_search, (any_fn)sfp8_sparse_linear_set_algo,
       (any_fn)sfp8_sparse_linear_get_algo, (any_fn)sfp8_sparse_linear_quant_workspace_bytes,
       (any_fn)sfp8_sparse_linear_quant, (any_fn)sfp8_sparse_linear_quant_host,
+      (any_fn)sfp8_sparse_linear_quant_fused, (any_fn)sfp8_sparse_linear_quant_chained,
+      (any_fn)sfp8_sparse_linear_quant_fusable,
       (any_fn)sfp8_sparse_linear_noalloc, (any_fn)sfp8_selftest_timeout,
       (any_fn)sfp8_read_device_status, (any_fn)sfp8_last_device_status,
       (any_fn)sfp8_compressed_values_bytes, (any_fn)sfp8_compressed_meta_bytes,
@@ -54,6 +56,11 @@ int main(void) {
       SFP8_ERR_UNSUPPORTED_DTYPE)
     return 10;
   if (sfp8_quantize_tensorwise_workspace_bytes((sfp8_amax_mode)7) != 0) return 11;
+  if (sfp8_sparse_linear_quant_fused(NULL, SFP8_E4M3, 128, SFP8_E4M3, NULL, NULL, 4, NULL,
+                                     SFP8_E4M3, NULL, 64, 128, NULL, NULL, NULL, 0, NULL) !=
+      SFP8_ERR_UNSUPPORTED_DTYPE)
+    return 12;
+  if (sfp8_sparse_linear_quant_fusable(16, 14336, 100) != 0) return 13;
 
   printf("abi ok\n");
   return 0;

@@ -156,22 +156,27 @@ def test_linear_validation_without_gpu(lib):
     assert na(FAKE, 0, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 4
     assert na(FAKE, 3, FAKE, 16, FAKE, 3, FAKE, 64, 0, None, FAKE, None) == 2
     assert na(FAKE, 3, FAKE, 0, FAKE, 3, FAKE, 64, 128, None, FAKE, None) == 0
-    fq = lib.sfp8_sparse_linear_quant
     qargs = [FAKE, 0, 128, 3, FAKE, FAKE, 16, FAKE, 3, FAKE, 64, 128, None, FAKE, FAKE,
              1 << 20, None]
+    for entry in ("sfp8_sparse_linear_quant", "sfp8_sparse_linear_quant_fused",
+                  "sfp8_sparse_linear_quant_chained"):
+        fq = getattr(lib, entry)
 
-    def qcall(**kw):
-        a = list(qargs)
-        names = ["x", "x_dt", "ld_x", "a_dt", "a_q", "s_a", "m", "packed", "w_dt", "s_w",
-                 "n", "k", "bias", "y", "ws", "wsb", "stream"]
-        for key, v in kw.items():
-            a[names.index(key)] = v
-        return fq(*a)
-    assert qcall(x_dt=3) == 4          # x must be bf16 / f16 / f32
-    assert qcall(ld_x=64) == 1         # ld_x < k
-    assert qcall(a_dt=0) == 4          # a_q must be FP8
-    assert qcall(k=192, ld_x=192) == 2
-    assert qcall(m=0) == 0
+        def qcall(**kw):
+            a = list(qargs)
+            names = ["x", "x_dt", "ld_x", "a_dt", "a_q", "s_a", "m", "packed", "w_dt", "s_w",
+                     "n", "k", "bias", "y", "ws", "wsb", "stream"]
+            for key, v in kw.items():
+                a[names.index(key)] = v
+            return fq(*a)
+        assert qcall(x_dt=3) == 4          # x must be bf16 / f16 / f32
+        assert qcall(ld_x=64) == 1         # ld_x < k
+        assert qcall(a_dt=0) == 4          # a_q must be FP8
+        assert qcall(k=192, ld_x=192) == 2
+        assert qcall(m=0) == 0
+    # host-only query: invalid sizes (and no device here) answer 0
+    assert lib.sfp8_sparse_linear_quant_fusable(16, 14336, 100) == 0
+    assert lib.sfp8_sparse_linear_quant_fusable(0, 14336, 4096) == 0
 
 
 @pytest.mark.parametrize("entry", ["sfp8_sparse_linear", "sfp8_sparse_linear_noalloc",
@@ -206,5 +211,40 @@ def test_linear_wrappers_reject_bad_arguments_without_gpu(lib, entry):
         call(out=torch.zeros((m, n + 1), dtype=torch.bfloat16))      # wrong shape
     with pytest.raises(ValueError, match="out"):
         call(out=torch.zeros((n, m), dtype=torch.bfloat16).t())      # not contiguous
+    with pytest.raises(ValueError, match="CUDA"):
+        call()                                                       # well-formed, on the CPU
+
+
+@pytest.mark.parametrize("entry", ["sfp8_sparse_linear_quant", "sfp8_sparse_linear_quant_fused",
+                                   "sfp8_sparse_linear_quant_chained"])
+def test_quant_wrappers_reject_bad_outputs_without_gpu(lib, entry):
+    """The one-call forward's wrappers check x, the bias and every output
+    tensor they are given (y, a_q, s_a) before any call reaches the library
+    (CPU tensors; nothing launches)."""
+    import torch
+    from semi_structured_sparse_rowwise_b200 import binding as B
+    m, n, k = 4, 64, 256
+    x = torch.zeros((m, k), dtype=torch.bfloat16)
+    s_w = torch.ones((n,), dtype=torch.float32)
+    packed = torch.zeros((16,), dtype=torch.uint8)
+    f = getattr(B, entry)
+
+    def call(x=x, **kw):
+        return f(x, "e4m3", packed, "e4m3", s_w, n, k, **kw)
+
+    with pytest.raises(ValueError, match="columns"):
+        call(x=torch.zeros((m, k - 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="dtype"):
+        call(x=torch.zeros((m, k), dtype=torch.int16))
+    with pytest.raises(ValueError, match="bias"):
+        call(bias=torch.zeros((n,), dtype=torch.float32))
+    with pytest.raises(ValueError, match="out"):
+        call(out=torch.zeros((m, n + 1), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="a_q"):
+        call(a_q=torch.zeros((m, k - 1), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="a_q"):
+        call(a_q=torch.zeros((m, 2 * k), dtype=torch.uint8)[:, :k])
+    with pytest.raises(ValueError, match="s_a"):
+        call(s_a=torch.zeros((m,), dtype=torch.float64))
     with pytest.raises(ValueError, match="CUDA"):
         call()                                                       # well-formed, on the CPU
