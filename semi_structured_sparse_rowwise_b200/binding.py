@@ -588,17 +588,19 @@ def sfp8_sparse_linear_quant_host(x_host, a_dtype, packed, w_dtype, s_w, n, k, x
     sparse linear, copy out, all on the current stream (page-locked host
     tensors keep it asynchronous).  Every buffer is given by the caller."""
     lib = load_library()
-    _require_cuda(x_dev, a_q, s_a, packed, s_w, bias, y_dev, workspace)
     if x_host.is_cuda or y_host.is_cuda:
         raise ValueError("x_host and y_host must be host tensors")
-    if not (x_host.is_contiguous() and y_host.is_contiguous() and x_dev.is_contiguous()):
-        raise ValueError("x_host, x_dev and y_host must be contiguous")
+    if not (x_host.is_contiguous() and y_host.is_contiguous() and x_dev.is_contiguous()
+            and y_dev.is_contiguous()):
+        raise ValueError("x_host, x_dev, y_dev and y_host must be contiguous")
     m = x_host.shape[0]
-    if x_host.shape != (m, k) or x_dev.shape != (m, k) or y_host.shape != (m, n):
-        raise ValueError("shapes: x_host/x_dev [m, k], y_host [m, n]")
+    if (x_host.shape != (m, k) or x_dev.shape != (m, k) or y_host.shape != (m, n)
+            or y_dev.shape != (m, n) or y_dev.dtype != torch.bfloat16):
+        raise ValueError("shapes: x_host/x_dev [m, k], y_host/y_dev [m, n] (y bfloat16)")
     xd = TORCH_WIDE.get(x_host.dtype)
     if xd is None or x_dev.dtype != x_host.dtype or y_host.dtype != torch.bfloat16:
         raise ValueError("x dtype bfloat16/float16/float32 (same on host and device), y bfloat16")
+    _require_cuda(x_dev, a_q, s_a, packed, s_w, bias, y_dev, workspace)
     dev = x_dev.device
     with torch.cuda.device(dev):
         st = lib.sfp8_sparse_linear_quant_host(

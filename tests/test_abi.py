@@ -248,3 +248,36 @@ def test_quant_wrappers_reject_bad_outputs_without_gpu(lib, entry):
         call(s_a=torch.zeros((m,), dtype=torch.float64))
     with pytest.raises(ValueError, match="CUDA"):
         call()                                                       # well-formed, on the CPU
+
+
+def test_host_wrapper_rejects_bad_buffers_without_gpu(lib):
+    """sfp8_sparse_linear_quant_host's wrapper checks the shapes, dtypes and
+    layout of its host and staging buffers before any call reaches the
+    library (CPU tensors; nothing launches)."""
+    import torch
+    from semi_structured_sparse_rowwise_b200 import binding as B
+    m, n, k = 4, 64, 256
+    bf = torch.bfloat16
+
+    def call(x_host=None, x_dev=None, y_dev=None, y_host=None):
+        return B.sfp8_sparse_linear_quant_host(
+            torch.zeros((m, k), dtype=bf) if x_host is None else x_host, "e4m3",
+            torch.zeros((16,), dtype=torch.uint8), "e4m3", torch.ones((n,)), n, k,
+            torch.zeros((m, k), dtype=bf) if x_dev is None else x_dev,
+            torch.zeros((m, k), dtype=torch.uint8), torch.ones((m,)),
+            torch.zeros((m, n), dtype=bf) if y_dev is None else y_dev,
+            torch.zeros((m, n), dtype=bf) if y_host is None else y_host,
+            torch.zeros((16,), dtype=torch.uint8))
+
+    with pytest.raises(ValueError, match="shapes"):
+        call(y_dev=torch.zeros((m, n + 1), dtype=bf))
+    with pytest.raises(ValueError, match="shapes"):
+        call(y_dev=torch.zeros((m, n), dtype=torch.float32))
+    with pytest.raises(ValueError, match="contiguous"):
+        call(y_dev=torch.zeros((n, m), dtype=bf).t())
+    with pytest.raises(ValueError, match="shapes"):
+        call(y_host=torch.zeros((m, n - 1), dtype=bf))
+    with pytest.raises(ValueError, match="dtype"):
+        call(x_host=torch.zeros((m, k), dtype=torch.float16))
+    with pytest.raises(ValueError, match="CUDA"):
+        call()                                                       # well-formed, on the CPU
