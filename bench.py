@@ -93,6 +93,12 @@ def kernel_source_sha1():
     return h.hexdigest()
 
 
+# Secondary roofline denominators: the datasheet figures (HBM3e 8 TB/s; FP8
+# with 2:4 sparsity 9 PFLOP/s dense-equivalent, at boost clock).
+DATASHEET_HBM_GBS = 8000.0
+DATASHEET_SPARSE_FP8_TFLOPS = 9000.0
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -126,8 +132,17 @@ class ClockSampler:
         self.reasons = set()
         self.max_mhz = None
         self._stop = threading.Event()
+        self._paused = threading.Event()
         self._thr = None
         self.ok = False
+
+    def pause(self):
+        """Stop sampling (host-only work in between: its idle clocks would
+        dilute the record)."""
+        self._paused.set()
+
+    def resume(self):
+        self._paused.clear()
 
     def __enter__(self):
         try:
@@ -158,10 +173,11 @@ class ClockSampler:
 
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self._sample()
-            except Exception:
-                pass
+            if not self._paused.is_set():
+                try:
+                    self._sample()
+                except Exception:
+                    pass
             time.sleep(self.period)
 
     def __exit__(self, *exc):
@@ -648,6 +664,10 @@ def run_ours(args):
         "roofline": {"bound": "tensor" if prefill else "hbm", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s" if prefill else "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
+                     "peak_datasheet": (DATASHEET_SPARSE_FP8_TFLOPS if prefill
+                                        else DATASHEET_HBM_GBS),
+                     "frac_datasheet": achieved / (DATASHEET_SPARSE_FP8_TFLOPS if prefill
+                                                   else DATASHEET_HBM_GBS),
                      "kernel": ("sparse_linear_pair_kernel" if m >= 512 else
                                 "sparse_linear_kernel"),
                      "algorithmic_bytes_per_launch": alg,
@@ -775,6 +795,8 @@ def prefill_case(args, S, synthetic, dev, bf16, capture, timed, shape_index, ste
                                   "replays against the sustained peak" % args.timed_seconds,
                         "achieved_sustained": tf, "peak_sustained": peak_sus,
                         "frac_sustained": tf / peak_sus, "unit": "TFLOP/s",
+                        "peak_datasheet": DATASHEET_SPARSE_FP8_TFLOPS,
+                        "frac_datasheet": tf_burst / DATASHEET_SPARSE_FP8_TFLOPS,
                         "traffic": traffic, "kernel": "sparse_linear_pair_kernel",
                         "algorithmic_flop_per_launch": flops},
            "clocks": clk.summary(), "clocks_burst": clk_burst.summary()}
@@ -897,12 +919,25 @@ def matrix_cases(args, workload, S, synthetic, dev, bf16, cases=None):
     table = []
     w_cache = {}
     inputs = {}
+    oracle_step_s = {}
     with ClockSampler(dev.index) as clk:
         for shape_index, a_fmt, w_fmt in cases:
             if shape_index not in inputs:
                 # the same seeded inputs serve every operand pair of a shape
                 inputs.clear()
                 inputs[shape_index] = synthetic.workload_inputs(workload, shape_index)
+                if not args.no_cpu_baseline:
+                    # the oracle on a bounded sample of this shape (host only)
+                    clk.pause()
+                    xb, wb = inputs[shape_index][0], inputs[shape_index][1]
+                    rows = min(64, xb.shape[0])
+                    rate, cores, note = oracle_prefill_rate(
+                        xb, wb, seconds=args.cpu_seconds_matrix, rows=rows, n_sample=512)
+                    m_, k_ = xb.shape
+                    oracle_step_s[shape_index] = (
+                        2.0 * m_ * wb.shape[0] * k_ / (rate * 1e12), cores,
+                        note if rows < m_ else note.replace("extrapolated", "sampled in N"))
+                    clk.resume()
             x_bits, w_bits, b_bits, seeds = inputs[shape_index]
             m, k = x_bits.shape
             n = w_bits.shape[0]
@@ -959,15 +994,25 @@ def matrix_cases(args, workload, S, synthetic, dev, bf16, cases=None):
             flops = 2.0 * m * n * k
             row = {"m": m, "k": k, "n": n, "a": a_fmt, "w": w_fmt, "bias": bias is not None,
                    "step_us": res["step"], "gemm_us": res["gemm"], "steps": steps}
+            cpu = oracle_step_s.get(shape_index)
             if m <= 128:
                 gbs = gemm_algorithmic_bytes(m, n, k) / (res["gemm"] * 1e-6) / 1e9
                 row.update({"bound": "hbm", "GB/s": gbs, "frac": gbs / hbm_peak,
+                            "frac_datasheet": gbs / DATASHEET_HBM_GBS,
                             "step_GB/s_weight": wbytes / (res["step"] * 1e-6) / 1e9})
+                if cpu is not None:
+                    row["cpu_baseline"] = {"value": wbytes / cpu[0] / 1e9,
+                                           "unit": "GB/s of compressed weight per step",
+                                           "cores": cpu[1], "kind": "oracle", "sample": cpu[2]}
             else:
                 tf = flops / (res["gemm"] * 1e-6) / 1e12
                 row.update({"bound": "tensor", "TFLOP/s": tf, "frac": tf / fl_peak,
                             "frac_sustained": tf / fl_sus,
+                            "frac_datasheet": tf / DATASHEET_SPARSE_FP8_TFLOPS,
                             "step_TFLOP/s": flops / (res["step"] * 1e-6) / 1e12})
+                if cpu is not None:
+                    row["cpu_baseline"] = {"value": flops / cpu[0] / 1e12, "unit": "TFLOP/s",
+                                           "cores": cpu[1], "kind": "oracle", "sample": cpu[2]}
             table.append(row)
             del x, ys, aq, sa, ws
     return table, clk.summary()
@@ -1002,9 +1047,13 @@ def run_matrix(args):
         "higher_is_better": True, "dtype": "fp8", "data": "synthetic",
         "config": {"workload": args.workload, "l2": "rotating >= 200 MB of compressed weight"},
         "peaks": {"hbm": [hbm_peak, hbm_kind], "tensor": [fl_peak, fl_kind],
-                  "tensor_sustained": [fl_sus, fl_sus_kind]},
+                  "tensor_sustained": [fl_sus, fl_sus_kind],
+                  "hbm_datasheet": DATASHEET_HBM_GBS,
+                  "sparse_fp8_datasheet": DATASHEET_SPARSE_FP8_TFLOPS},
         "table": table, "clocks": clocks,
     }
+    if "cpu_baseline" in big:
+        line["cpu_baseline"] = big["cpu_baseline"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -1033,6 +1082,8 @@ def main():
     ap.add_argument("--all-m", action="store_true", help="also time M=1 and M=4")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds-matrix", type=float, default=1.0,
+                    help="seconds of oracle work per shape of the sweep and stress tables")
     ap.add_argument("--cpu-seconds-prefill", type=float, default=3.0,
                     help="oracle seconds per prefill shape in the default run")
     ap.add_argument("--replays", type=int, default=0,
