@@ -36,3 +36,62 @@ def test_parser_accepts_every_mode():
     for mode in ("decode_gate_up_8b", "prefill_8b", "quantize_tensorwise", "dtype_sweep_8b_up",
                  "stress_70b_mlp"):
         assert mode in r.stdout
+
+
+class _FakeNvml:
+    """Stands in for pynvml: a clock the test sets and a power-cap reason."""
+    NVML_CLOCK_SM = 0
+
+    def __init__(self):
+        self.mhz = 1965
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.mhz
+
+    def nvmlDeviceGetCurrentClocksThrottleReasons(self, h):
+        return 0x4          # sw_power_cap
+
+
+def test_clock_sampler_pause_keeps_host_only_time_out(monkeypatch):
+    """Samples taken while paused (host-only work, idle GPU clocks) must not
+    enter the record; the throttle reasons are named."""
+    import time
+    fake = _FakeNvml()
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    with bench.ClockSampler(0, period_s=0.001) as clk:
+        time.sleep(0.05)
+        clk.pause()
+        n_before = len(clk.samples)
+        fake.mhz = 345                      # what an idle GPU would report
+        time.sleep(0.05)
+        n_paused = len(clk.samples)
+        fake.mhz = 1965
+        clk.resume()
+        time.sleep(0.05)
+    s = clk.summary()
+    assert n_before > 0
+    assert n_paused <= n_before + 1          # at most one sample already in flight
+    assert 345 not in clk.samples[n_before + 1:]
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == len(clk.samples)
+
+
+def test_oracle_sample_extrapolates_linearly():
+    """The oracle baseline on a bounded sample: a positive dense-equivalent
+    rate, labelled as extrapolated from the rows and columns it timed."""
+    from semi_structured_sparse_rowwise_b200 import synthetic
+    x = synthetic.activation(11, 8, 256)
+    w = synthetic.weight(12, 96, 256)
+    rate, cores, note = bench.oracle_prefill_rate(x, w, seconds=0.05, rows=4, n_sample=32)
+    assert rate > 0 and cores >= 1
+    assert note.startswith("extrapolated") and "4 of 8 activation rows" in note
+    assert "32 of 96 output columns" in note
