@@ -152,6 +152,14 @@ def _require_cuda(*ts):
             raise ValueError("tensors must be CUDA tensors")
 
 
+def _ws_bytes(ws, device):
+    """Size in bytes of a caller's workspace (any dtype), which must be a
+    contiguous CUDA tensor on `device`."""
+    if not ws.is_cuda or ws.device != torch.device(device) or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor on %s" % (device,))
+    return ws.numel() * ws.element_size()
+
+
 def sfp8_quantize_rowwise(x, q_dtype="e4m3", q=None, scales=None):
     """x [rows, cols] bf16/f16/f32 (unit column stride) -> (q uint8, scales f32)."""
     lib = load_library()
@@ -209,7 +217,8 @@ def sfp8_quantize_tensorwise(x, q_dtype="e4m3", mode="reduce", q=None, scale=Non
     with torch.cuda.device(x.device):
         st = lib.sfp8_quantize_tensorwise(_ptr(x), DTYPE[xd], x.numel(), _ptr(q),
                                           DTYPE[_fp8_name(q_dtype)], _ptr(scale),
-                                          AMAX_MODE[mode], _ptr(workspace), workspace.numel(),
+                                          AMAX_MODE[mode], _ptr(workspace),
+                                          _ws_bytes(workspace, x.device),
                                           _stream(x.device))
     _check(st, "sfp8_quantize_tensorwise")
     return q, scale
@@ -310,7 +319,7 @@ def new_workspace(m, n, k, device):
 def sfp8_workspace_clear(workspace):
     lib = load_library()
     with torch.cuda.device(workspace.device):
-        st = lib.sfp8_workspace_clear(_ptr(workspace), workspace.numel(),
+        st = lib.sfp8_workspace_clear(_ptr(workspace), _ws_bytes(workspace, workspace.device),
                                       _stream(workspace.device))
     _check(st, "sfp8_workspace_clear")
 
@@ -347,7 +356,7 @@ def sfp8_sparse_linear(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bias=None,
         st = lib.sfp8_sparse_linear(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
                                     _ptr(packed), DTYPE[_fp8_name(w_dtype)],
                                     _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
-                                    workspace.numel(), _stream(a_q.device))
+                                    _ws_bytes(workspace, a_q.device), _stream(a_q.device))
     _check(st, "sfp8_sparse_linear")
     return out
 
@@ -435,7 +444,7 @@ def sfp8_sparse_linear_algo(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, algo,
         st = lib.sfp8_sparse_linear_algo(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
                                          _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n,
                                          k, _ptr(bias), _ptr(out), algo, _ptr(workspace),
-                                         workspace.numel(), _stream(a_q.device))
+                                         _ws_bytes(workspace, a_q.device), _stream(a_q.device))
     _check(st, "sfp8_sparse_linear_algo")
     return out
 
@@ -459,7 +468,8 @@ def sfp8_sparse_linear_search(a_q, a_dtype, s_a, packed, w_dtype, s_w, n, k, bia
         st = lib.sfp8_sparse_linear_search(_ptr(a_q), DTYPE[_fp8_name(a_dtype)], _ptr(s_a), m,
                                            _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w),
                                            n, k, _ptr(bias), _ptr(out), _ptr(ws), ws.numel(),
-                                           _ptr(flush), 0 if flush is None else flush.numel(),
+                                           _ptr(flush),
+                                           0 if flush is None else _ws_bytes(flush, dev),
                                            reps, ctypes.byref(best), times, count, _stream(dev))
     _check(st, "sfp8_sparse_linear_search")
     return int(best.value), [float(t) for t in times[:count]]
@@ -567,7 +577,7 @@ def _quant_linear(name, x, a_dtype, packed, w_dtype, s_w, n, k, bias, out, works
         st = getattr(lib, name)(_ptr(x), DTYPE[xd], ld, DTYPE[_fp8_name(a_dtype)], _ptr(a_q),
                                 _ptr(s_a), m, _ptr(packed), DTYPE[_fp8_name(w_dtype)],
                                 _ptr(s_w), n, k, _ptr(bias), _ptr(out), _ptr(workspace),
-                                workspace.numel(), _stream(dev))
+                                _ws_bytes(workspace, dev), _stream(dev))
     _check(st, name)
     return out, a_q, s_a
 
@@ -606,7 +616,7 @@ def sfp8_sparse_linear_quant_host(x_host, a_dtype, packed, w_dtype, s_w, n, k, x
         st = lib.sfp8_sparse_linear_quant_host(
             _ptr(x_host), _ptr(x_dev), DTYPE[xd], DTYPE[_fp8_name(a_dtype)], _ptr(a_q), _ptr(s_a),
             m, _ptr(packed), DTYPE[_fp8_name(w_dtype)], _ptr(s_w), n, k, _ptr(bias), _ptr(y_dev),
-            _ptr(y_host), _ptr(workspace), workspace.numel(), _stream(dev))
+            _ptr(y_host), _ptr(workspace), _ws_bytes(workspace, dev), _stream(dev))
     _check(st, "sfp8_sparse_linear_quant_host")
     return y_host
 

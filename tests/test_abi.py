@@ -281,3 +281,17 @@ def test_host_wrapper_rejects_bad_buffers_without_gpu(lib):
         call(x_host=torch.zeros((m, k), dtype=torch.float16))
     with pytest.raises(ValueError, match="CUDA"):
         call()                                                       # well-formed, on the CPU
+
+
+def test_workspace_size_is_counted_in_bytes():
+    """A caller's workspace of any dtype is passed as its size in bytes; a
+    non-contiguous or CPU workspace is refused before any call."""
+    import torch
+    from semi_structured_sparse_rowwise_b200 import binding as B
+    with pytest.raises(ValueError, match="workspace"):
+        B._ws_bytes(torch.zeros((64,), dtype=torch.uint8), "cpu")
+    if torch.cuda.is_available():
+        w = torch.zeros((16,), dtype=torch.float32, device="cuda")
+        assert B._ws_bytes(w, w.device) == 64
+        with pytest.raises(ValueError, match="workspace"):
+            B._ws_bytes(torch.zeros((8, 8), device="cuda").t(), w.device)
