@@ -311,6 +311,36 @@ def oracle_prefill_rate(x_bits, w_bits, seconds=3.0, rows=64, n_sample=1024):
     return rate, cores, note
 
 
+def oracle_offline_time(w_bits, seconds=2.0, n_sample=256):
+    """Oracle time of the offline weight preparation on a bounded sample:
+    prune (bf16), row-wise quantise and compress n_sample weight rows,
+    repeated for about `seconds`, scaled to all rows.  Returns (seconds for
+    the whole weight, cores, note)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    n, k = w_bits.shape
+    rows = min(n_sample, n)
+    w32 = oracle.bf16_bits_to_f32(w_bits[:rows])
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        wq, sw = oracle.quantize_rowwise(oracle.prune_24(w32), "e4m3")
+        oracle.compress_24(wq, "e4m3")
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    t_full = dt / reps * (n / rows)
+    note = ("extrapolated: oracle prune + row-wise quantise + compress of %d of %d weight rows "
+            "(k = %d), %d repetitions in %.1f s, scaled linearly to all rows; %d BLAS threads"
+            % (rows, n, k, reps, dt, cores))
+    return t_full, cores, note
+
+
 def run_reference(args):
     rank, local, world = dist_setup("gloo")
     if rank != 0:
@@ -698,6 +728,13 @@ def run_ours(args):
             rate, cores, note, _ = oracle_step_rate(m, seconds=args.cpu_seconds)
             line["cpu_baseline"] = {"value": rate, "unit": "GB/s", "cores": cores,
                                     "kind": "oracle", "sample": note}
+            # the offline weight preparation, beside the GPU's "prepare_weight_24"
+            # (the same algorithmic bytes: bf16 weight in, packed weight and scales out)
+            t_prep, cores, note = oracle_offline_time(w_bits, seconds=2.0)
+            line["offline_cpu_baseline"] = {
+                "value": (n * k * 2 + compressed_weight_bytes(n, k) + 4 * n) / t_prep / 1e9,
+                "unit": "GB/s", "ms": t_prep * 1e3, "cores": cores, "kind": "oracle",
+                "sample": note}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_step, g_gemm, g_q

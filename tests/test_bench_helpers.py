@@ -95,3 +95,13 @@ def test_oracle_sample_extrapolates_linearly():
     assert rate > 0 and cores >= 1
     assert note.startswith("extrapolated") and "4 of 8 activation rows" in note
     assert "32 of 96 output columns" in note
+
+
+def test_oracle_offline_sample_scales_to_all_rows():
+    """The offline oracle baseline (prune + quantise + compress) on a sample
+    of rows: a positive time for the whole weight, labelled as extrapolated."""
+    from semi_structured_sparse_rowwise_b200 import synthetic
+    w = synthetic.weight(13, 64, 256)
+    t, cores, note = bench.oracle_offline_time(w, seconds=0.05, n_sample=16)
+    assert t > 0 and cores >= 1
+    assert note.startswith("extrapolated") and "16 of 64 weight rows" in note
