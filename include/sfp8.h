@@ -420,8 +420,9 @@ size_t sfp8_sparse_linear_quant_workspace_bytes(int64_t m, int64_t n, int64_t k)
  *  packed, w_dtype, s_w, n, k, bias, y: as for sfp8_sparse_linear.
  *  workspace  >= sfp8_sparse_linear_quant_workspace_bytes(m, n, k) bytes,
  *          zero before the first call (left zero by every call).
- *  x must not overlap a_q, s_a or y (the fused kernel reads x in every CTA
- *  while some CTAs already write a_q and s_a).
+ *  x's span (rows 0..m-1 at stride ld_x) must not overlap a_q, s_a or y (the
+ *  kernels read x while they write those); with n > 0 an overlap is refused
+ *  with SFP8_ERR_INVALID_ARG before anything is launched.
  *
  * Returns the first failing status of the two steps (validation of both
  * before anything is launched where the arguments allow).  With n == 0 only

@@ -664,12 +664,44 @@ sfp8_status encode_y_2d(CUtensorMap* map, void* y, uint64_t m, uint64_t n, uint3
 }
 
 
+// Whether x [m rows of ld_x elements, k used] shares bytes with a_q [m, k],
+// s_a [m] or y [m, n] bf16 (host arithmetic on the addresses; sizes that do
+// not fit are left to the size checks that follow).  The quantiser reads x
+// while it writes a_q and s_a, and the fused GEMM reads x in every CTA while
+// some CTAs already write.
+bool outputs_overlap_input(const void* x, sfp8_dtype x_dtype, int64_t ld_x, int64_t m,
+                                  int64_t k, const void* a_q, const void* s_a, const void* y,
+                                  int64_t n) {
+  const int64_t lim = int64_t(1) << 31;
+  if (x == nullptr || m <= 0 || k <= 0 || m >= lim || k >= lim || n < 0 || n >= lim) return false;
+  int64_t span = 0;
+  if (__builtin_mul_overflow(m - 1, ld_x, &span) || __builtin_add_overflow(span, k, &span) ||
+      __builtin_mul_overflow(span, static_cast<int64_t>(elem_size(x_dtype)), &span))
+    return false;
+  const uintptr_t xb = reinterpret_cast<uintptr_t>(x);
+  const uintptr_t xe = xb + static_cast<uintptr_t>(span);
+  auto hits = [&](const void* p, int64_t bytes) {
+    if (p == nullptr || bytes <= 0) return false;
+    const uintptr_t b = reinterpret_cast<uintptr_t>(p);
+    return b < xe && xb < b + static_cast<uintptr_t>(bytes);
+  };
+  return hits(a_q, m * k) || hits(s_a, 4 * m) || hits(y, 2 * m * n);
+}
+
+// The activation that the one-call forward reads (for the overlap check).
+struct XSpan {
+  const void* x;
+  sfp8_dtype dtype;
+  int64_t ld;
+};
+
 // Validation shared by the sparse-linear entry points (everything except the
-// workspace); on success fills *plan for the current device.
+// workspace); on success fills *plan for the current device.  With `xs`
+// (the one-call forward), outputs sharing bytes with x are refused too.
 sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_a, int64_t m,
                             const void* packed, sfp8_dtype w_dtype, const float* s_w, int64_t n,
                             int64_t k, const void* bias, const void* y, DeviceInfo** dev,
-                            LinearPlan* plan, bool* empty) {
+                            LinearPlan* plan, bool* empty, const XSpan* xs = nullptr) {
   *empty = false;
   if (!is_fp8(a_dtype) || !is_fp8(w_dtype)) return SFP8_ERR_UNSUPPORTED_DTYPE;
   if (m < 0 || n < 0 || k < 0) return SFP8_ERR_INVALID_ARG;
@@ -685,6 +717,8 @@ sfp8_status validate_linear(const void* a_q, sfp8_dtype a_dtype, const float* s_
   if (!aligned(a_q, 16) || !aligned(packed, 16) || !aligned(s_a, 4) || !aligned(s_w, 4) ||
       !aligned(y, 2) || (bias != nullptr && !aligned(bias, 2)))
     return SFP8_ERR_MISALIGNED;
+  if (xs != nullptr && outputs_overlap_input(xs->x, xs->dtype, xs->ld, m, k, a_q, s_a, y, n))
+    return SFP8_ERR_INVALID_ARG;
   sfp8_status s = current_device(dev);
   if (s != SFP8_OK) return s;
   *plan = make_plan((*dev)->index, m, n, k, (*dev)->num_sms);
@@ -1493,8 +1527,9 @@ static sfp8_status quant_linear(const void* x, sfp8_dtype x_dtype, int64_t ld_x,
   DeviceInfo* dev = nullptr;
   LinearPlan pl{};
   bool empty = false;
+  const XSpan xs{x, x_dtype, ld_x};
   sfp8_status s = validate_linear(a_q, a_dtype, s_a, m, packed, w_dtype, s_w, n, k, bias, y,
-                                  &dev, &pl, &empty);
+                                  &dev, &pl, &empty, &xs);
   if (s != SFP8_OK) return s;
   if (m > 0 && x == nullptr) return SFP8_ERR_INVALID_ARG;
   const int es = elem_size(x_dtype);

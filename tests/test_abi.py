@@ -295,3 +295,30 @@ def test_workspace_size_is_counted_in_bytes():
         assert B._ws_bytes(w, w.device) == 64
         with pytest.raises(ValueError, match="workspace"):
             B._ws_bytes(torch.zeros((8, 8), device="cuda").t(), w.device)
+
+
+@pytest.mark.parametrize("entry", ["sfp8_sparse_linear_quant", "sfp8_sparse_linear_quant_fused",
+                                   "sfp8_sparse_linear_quant_chained"])
+def test_quant_entry_points_refuse_outputs_overlapping_x(lib, entry):
+    """x is read while a_q, s_a and y are written: an output sharing bytes
+    with x's span (rows 0..m-1 at stride ld_x) is refused with
+    SFP8_ERR_INVALID_ARG before any device is touched; disjoint buffers pass
+    on to the device checks (no device here: SFP8_ERR_CUDA or _ARCH)."""
+    f = getattr(lib, entry)
+    X = 0x100000
+    m, k, n = 16, 256, 64
+
+    def call(a_q, s_a, y, ld=k):
+        return f(ctypes.c_void_p(X), 0, ld, 3, ctypes.c_void_p(a_q), ctypes.c_void_p(s_a), m,
+                 ctypes.c_void_p(0x900000), 3, ctypes.c_void_p(0xA00000), n, k, None,
+                 ctypes.c_void_p(y), ctypes.c_void_p(0xB00000), 1 << 20, None)
+    x_end = X + m * k * 2
+    assert call(0x200000, 0x300000, 0x400000) in (5, 7)              # disjoint
+    assert call(X + 256, 0x300000, 0x400000) == 1                    # a_q inside x
+    assert call(0x200000, x_end - 4, 0x400000) == 1                  # s_a's first bytes in x
+    assert call(0x200000, x_end, 0x400000) in (5, 7)                 # s_a right after x
+    assert call(0x200000, 0x300000, X - m * n * 2 + 2) == 1          # y's last bytes in x
+    assert call(0x200000, 0x300000, X - m * n * 2) in (5, 7)         # y right before x
+    # x with row stride 512: its span ends with row 15's 256 values (X + 15872)
+    assert call(X + 14 * 1024 + 512, 0x300000, 0x400000, ld=512) == 1   # inside the span
+    assert call(X + 15 * 1024 + 512, 0x300000, 0x400000, ld=512) in (5, 7)   # right after it
